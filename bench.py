@@ -1,0 +1,413 @@
+#!/usr/bin/env python
+"""Benchmark of the sparse MoE FFN forward layer (router + dispatch + routed SwiGLU
+experts + weighted combine + shared expert) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one whole layer call (moe_router then moe_forward) on one batch of
+seeded synthetic inputs shaped like the workload, inputs already in HBM.  With
+N > 1 (launched by torchrun, one rank per GPU) every rank runs its own replica
+on its own batch (tokens are independent, no collective on the data path); the
+step time is the max over ranks and `value` counts the tokens of all ranks.
+Rank 0 prints one JSON line.  `--impl reference` times the plain fp64 CPU oracle
+on the same workload instead (the reference arm of this comparison).
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from workloads import CONFIGS, DEFAULT_WORKLOAD, make_inputs  # noqa: E402
+
+METRIC = "MoE-layer tokens/s (prefill, decode) and % of bf16 tensor / HBM roofline"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+BF16_KERNELS = ["dispatch_count", "dispatch_scan", "dispatch_scatter", "dispatch_gather",
+                "gate_up_swiglu", "down_combine_shared"]
+F32_KERNELS = ["dispatch_count", "dispatch_scan", "dispatch_scatter", "gate_up_routed",
+               "gate_up_shared", "down_routed", "down_shared", "combine"]
+KERNEL_SOURCES = {
+    "gate_up_swiglu": "sparse_moe_layer_02_b200/csrc/gemm_sm100.cuh",
+    "down_combine_shared": "sparse_moe_layer_02_b200/csrc/gemm_sm100.cuh",
+    "router": "sparse_moe_layer_02_b200/csrc/router.cuh",
+}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="target duration of the oracle's CPU-baseline sample")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in FALLBACK_PEAKS}, "measured"
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+
+    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.dev = device_index
+        self.path = None
+
+    def start(self):
+        try:
+            import tempfile
+            fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+            os.close(fd)
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), "--query-gpu=" + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.out, stderr=subprocess.DEVNULL)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) == len(self.FIELDS):
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[4 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def source_sha(rel: str) -> str:
+    with open(os.path.join(ROOT, rel), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def stored_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel is unchanged."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)
+        rec = t[kernel][workload]
+        if rec.get("source_sha") != source_sha(KERNEL_SOURCES[kernel]):
+            return None
+        return float(rec["bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
+def kernel_work(cfg, name: str, hit: int):
+    """Algorithmic FLOPs and bytes of one launch (routed k experts, shared expert,
+    router; weights of hit experts read once, x read once, y written once)."""
+    es = 2 if cfg.dtype == torch.bfloat16 else 4
+    ws = 2 if cfg.wg_dtype == torch.bfloat16 else 4
+    N, D, E, k, d, dsh = cfg.N, cfg.D, cfg.E, cfg.k, cfg.d_moe, cfg.d_sh
+    if name == "gate_up_swiglu":
+        flops = 2.0 * (N * k * 2 * d + N * 2 * dsh) * D
+        byts = (hit * 2 * d + 2 * dsh) * D * es + N * D * es
+    elif name == "down_combine_shared":
+        flops = 2.0 * (N * k * d + N * dsh) * D
+        byts = (hit * d + dsh) * D * es + N * D * es
+    elif name == "router":
+        flops = 2.0 * N * D * E
+        byts = E * D * ws + N * D * es
+    else:
+        flops, byts = 0.0, 0.0
+    return flops, byts
+
+
+def oracle_time(cfg, inp_host, n_tokens: int, target_s: float, max_reps: int = 50):
+    """Run the oracle (router + forward) on the first n_tokens of the batch until
+    target_s has elapsed; returns (tokens/s, tokens, seconds, reps)."""
+    import oracle
+
+    x = inp_host.x[:n_tokens].contiguous()
+    done, t0, reps = 0, time.perf_counter(), 0
+    while True:
+        r = oracle.router(x, inp_host.W_g, inp_host.b, cfg.n_group, cfg.topk_group, cfg.k,
+                          cfg.norm_topk_prob, cfg.alpha)
+        oracle.forward(x, inp_host.gate_up, inp_host.down, inp_host.sh_gate, inp_host.sh_up,
+                       inp_host.sh_down, r["idx"], r["w"])
+        done += n_tokens
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= target_s or reps >= max_reps:
+            return done / el, done, el, reps
+
+
+def run_reference(args):
+    """Reference arm: the fp64 CPU oracle on the same workload, rank 0 only."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+
+    cfg = CONFIGS[args.workload]
+    gen_dev = "cuda:0" if torch.cuda.is_available() else "cpu"
+    inp = make_inputs(cfg, seed=0, device=gen_dev).to("cpu")
+    cores = oracle.num_threads()
+    # Size each step's sample so that warm-up + timed steps end within ~2 minutes.
+    _, _, t1, _ = oracle_time(cfg, inp, min(cfg.N, cores), 0.0, max_reps=1)
+    per_tok = t1 / min(cfg.N, cores)
+    budget = 120.0 / max(args.steps + args.warmup, 1)
+    sample = int(max(1, min(cfg.N, budget / max(per_tok, 1e-9))))
+    x = inp.x[:sample].contiguous()
+
+    def step():
+        r = oracle.router(x, inp.W_g, inp.b, cfg.n_group, cfg.topk_group, cfg.k,
+                          cfg.norm_topk_prob, cfg.alpha)
+        oracle.forward(x, inp.gate_up, inp.down, inp.sh_gate, inp.sh_up, inp.sh_down, r["idx"],
+                       r["w"])
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    el = time.perf_counter() - t0
+    value = sample * args.steps / el
+    desc = "fp64 oracle (router + forward) on the first %d of %d tokens of %s per step" % (
+        sample, cfg.N, cfg.name)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": cfg.name, "description": cfg.description, "N": cfg.N,
+                       "D": cfg.D, "E": cfg.E, "k": cfg.k, "d_moe": cfg.d_moe,
+                       "sample_tokens_per_step": sample},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    import sparse_moe_layer_02_b200 as moe
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    cfg = CONFIGS[args.workload]
+    inp = make_inputs(cfg, seed=0, device=dev)
+    if rank > 0:  # each replica gets its own batch of tokens
+        from workloads import make_tokens
+        inp.x = make_tokens(cfg, cfg.N, seed=1000 + rank, device=dev)
+    N, D = cfg.N, cfg.D
+    ws = torch.empty(max(moe.moe_forward_workspace(N, D, cfg.E, cfg.d_moe, cfg.d_sh, cfg.k,
+                                                   cfg.dtype), 256), dtype=torch.uint8, device=dev)
+    y = torch.empty((N, D), dtype=cfg.dtype, device=dev)
+    idx = torch.empty((N, cfg.k), dtype=torch.int32, device=dev)
+    w = torch.empty((N, cfg.k), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    kernels = BF16_KERNELS if cfg.dtype == torch.bfloat16 else F32_KERNELS
+
+    def step(x):
+        moe.moe_router(x, inp.W_g, inp.b, cfg.n_group, cfg.topk_group, cfg.k, cfg.norm_topk_prob,
+                       cfg.alpha, idx, w, stream)
+        moe.moe_forward(x, inp.gate_up, inp.down, inp.sh_gate, inp.sh_up, inp.sh_down, idx, w, y,
+                        ws, stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step(inp.x)
+    status = moe.moe_device_status(stream)
+    if status != 0:
+        raise SystemExit("device status after warm-up: %s" % moe.moe_status_string(status))
+    loads = torch.bincount(idx.flatten().long(), minlength=cfg.E)
+    hit = int((loads > 0).sum().item())
+    max_over_mean = float(loads.max().item() / loads.float().mean().item())
+
+    # Per-step events: router start/end, then moe_forward's kernel boundaries.
+    K = args.steps
+    nk = len(kernels)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 2)] for _ in range(K)]
+    for row in evs:  # create the underlying CUDA events
+        for e in row:
+            e.record(stream)
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local)
+    sampler.start()
+    launches0 = moe.moe_launch_count()
+    start.record(stream)
+    for s in range(K):
+        row = evs[s]
+        row[0].record(stream)
+        moe.moe_router(inp.x, inp.W_g, inp.b, cfg.n_group, cfg.topk_group, cfg.k,
+                       cfg.norm_topk_prob, cfg.alpha, idx, w, stream)
+        moe.moe_profile_set_events(row[1:])
+        moe.moe_forward(inp.x, inp.gate_up, inp.down, inp.sh_gate, inp.sh_up, inp.sh_down, idx, w,
+                        y, ws, stream)
+    end.record(stream)
+    end.synchronize()
+    launches = moe.moe_launch_count() - launches0
+    moe.moe_profile_set_events([])
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    status = moe.moe_device_status(stream)
+    if status != 0:
+        raise SystemExit("device status after timing: %s" % moe.moe_status_string(status))
+    total_ms = start.elapsed_time(end)
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if dist:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+    ms_per_step = total_ms / K
+    value = N * world * K / (total_ms / 1e3)
+
+    # Per-kernel durations over the timed region.
+    per = {"router": sum(evs[s][0].elapsed_time(evs[s][1]) for s in range(K)) / K}
+    for i, name in enumerate(kernels):
+        per[name] = sum(evs[s][1 + i].elapsed_time(evs[s][2 + i]) for s in range(K)) / K
+    dom = max(per, key=per.get)
+    peaks, peak_src = load_peaks()
+    flops, byts = kernel_work(cfg, dom, hit)
+    dur_s = per[dom] / 1e3
+    ridge = peaks["bf16_tflops_sustained"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    if byts > 0 and flops / byts < ridge:
+        roof = {"bound": "hbm", "achieved": byts / dur_s / 1e9, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s"}
+    else:
+        roof = {"bound": "tensor", "achieved": flops / dur_s / 1e12,
+                "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"] if roof["peak"] else None
+    roof["traffic"] = stored_traffic(dom, cfg.name) if dom in KERNEL_SOURCES else None
+    roof["kernel"] = dom
+    roof["peak_source"] = peak_src + (" sustained bf16" if roof["bound"] == "tensor" else " copy")
+    roof["ms_per_launch"] = per[dom]
+    roof["algorithmic"] = {"flops": flops, "bytes": byts}
+
+    # End to end: pinned host x in, layer, pinned host y out, all inside the timed region.
+    x_host = inp.x.cpu().pin_memory()
+    y_host = torch.empty((N, D), dtype=cfg.dtype).pin_memory()
+    x_dev = torch.empty_like(inp.x)
+    for _ in range(3):
+        x_dev.copy_(x_host, non_blocking=True)
+        step(x_dev)
+        y_host.copy_(y, non_blocking=True)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(K):
+        x_dev.copy_(x_host, non_blocking=True)
+        step(x_dev)
+        y_host.copy_(y, non_blocking=True)
+    e1.record(stream)
+    e1.synchronize()
+    et = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if dist:
+        dist.all_reduce(et, op=dist.ReduceOp.MAX)
+    e2e_value = N * world * K / (float(et.item()) / 1e3)
+    es = inp.x.element_size()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+
+        host = inp.to("cpu")
+        n = min(cfg.N, 32)
+        v, done, el, reps = oracle_time(cfg, host, n, args.cpu_seconds)
+        cpu = {"value": v, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+               "sample": "fp64 oracle router + forward on the first %d tokens of the %d-token "
+                         "batch, %d repetitions, %.1f s" % (n, cfg.N, reps, el)}
+
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if cfg.dtype == torch.bfloat16 else "f32", "data": "synthetic",
+        "config": {"workload": cfg.name, "description": cfg.description, "N": N, "D": D,
+                   "E": cfg.E, "n_group": cfg.n_group, "topk_group": cfg.topk_group, "k": cfg.k,
+                   "d_moe": cfg.d_moe, "d_sh": cfg.d_sh, "alpha": cfg.alpha,
+                   "router_dtype": str(cfg.wg_dtype).replace("torch.", ""),
+                   "hit_experts": hit, "max_over_mean_load": max_over_mean,
+                   "parallelism": "replicas" if world > 1 else "single",
+                   "l2": "inputs larger than L2 (hit-expert weights %.2f GB per step)"
+                         % (kernel_work(cfg, "gate_up_swiglu", hit)[1] / 1e9
+                            + kernel_work(cfg, "down_combine_shared", hit)[1] / 1e9)},
+        "roofline": roof,
+        "kernel_ms": per,
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": N * D * es,
+                "d2h_bytes_per_step": N * D * es},
+        "gpu_launches": int(launches),
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

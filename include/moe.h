@@ -1,0 +1,158 @@
+/*
+ * moe.h — C ABI of the B200 (sm_100a) sparse mixture-of-experts FFN forward
+ * (GLM-4.5 / GLM-5 style): a sigmoid router with a loss-free correction bias and
+ * group-restricted top-k, token dispatch, routed SwiGLU experts, a
+ * routing-weighted combine and an always-on shared expert:
+ *
+ *     y_n = sum_{i in T(n)} w_{n,i} E_i(x_n) + E_sh(x_n)
+ *
+ * Conventions for every entry point
+ *   - All tensor pointers are DEVICE pointers to caller-owned, contiguous,
+ *     row-major memory.  The library never allocates, frees or retains them.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Calls only enqueue work and return; results are ready when the stream is.
+ *   - Argument and shape errors are reported synchronously, before any launch;
+ *     nothing is written then.  Launch failures return MOE_ERR_CUDA.  Errors
+ *     found by the kernels themselves (an out-of-range expert id, a bounded wait
+ *     that ran out) are recorded in a device status word that
+ *     moe_device_status() reads.
+ *   - Pointers must be 16-byte aligned.  For bf16 tensors the row lengths D,
+ *     d_moe and d_sh must be multiples of 8 (16-byte rows for TMA).
+ *   - Calls on one device may overlap only if they are on one stream: the
+ *     kernels share nothing across calls except the status word, but two
+ *     moe_forward calls must not share a workspace while both are in flight.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Element types of the tensors handed across the boundary. */
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_ARG = -1,            /* null pointer, misaligned pointer, bad flag */
+    MOE_ERR_SHAPE = -2,          /* inconsistent or unsupported sizes */
+    MOE_ERR_DTYPE = -3,          /* unsupported dtype combination */
+    MOE_ERR_WORKSPACE = -4,      /* workspace missing or smaller than required */
+    MOE_ERR_CUDA = -5,           /* a CUDA runtime call or launch failed */
+    MOE_ERR_DEVICE_TIMEOUT = -6, /* a bounded device-side wait ran out */
+    MOE_ERR_BAD_INDEX = -7,      /* topk_idx held an id outside [0, E]; skipped */
+    MOE_ERR_NO_DEVICE = -8       /* no sm_100 device is current */
+} moe_status;
+
+/*
+ * moe_router — group-restricted sigmoid router.
+ * Defined by "GLM-4.5 Group Router", How it works: r = x W_g^T in float32,
+ * s = sigmoid(r), s' = s + b (the correction bias is used for selection only),
+ * the E experts form n_group contiguous groups of E/n_group, a group scores the
+ * sum of its two largest s', the topk_group best groups are kept, T = the k
+ * largest s' inside them, and w_i = alpha * s_i / (sum_{j in T} s_j + 1e-20)
+ * when norm_topk_prob (else alpha * s_i).  n_group = topk_group = 1 is plain
+ * top-k.  alpha is applied here and nowhere else ("GLM-4.5 MoE Forward",
+ * note on applying routed_scaling_factor once).
+ *
+ *   x        [N, D]   x_dtype (MOE_F32 or MOE_BF16)
+ *   W_g      [E, D]   wg_dtype (MOE_F32 or MOE_BF16)
+ *   b        [E]      fp32 correction bias
+ *   topk_idx [N, k]   int32 out: expert ids, ordered by descending s', ties to
+ *                     the lower id; never the sentinel E
+ *   topk_w   [N, k]   fp32 out: mixture weights matching topk_idx, alpha included
+ * Sizes: 1 <= E <= 512, E % n_group == 0, E / n_group >= 2 when n_group > 1,
+ * 1 <= topk_group <= n_group, 1 <= k <= min(32, topk_group * E / n_group),
+ * n_group <= 64, D >= 1.  N = 0 is a no-op.
+ * Logits accumulate in fp32 (bf16 x bf16 and bf16 x fp32 products are exact in
+ * fp32), so ids agree with an exact evaluation except where two candidates'
+ * s' lie within fp32 rounding of each other.
+ */
+int moe_router(const void *x, int x_dtype, const void *W_g, int wg_dtype, const float *b,
+               int N, int D, int E, int n_group, int topk_group, int k, int norm_topk_prob,
+               float alpha, int32_t *topk_idx, float *topk_w, void *stream);
+
+/*
+ * moe_forward_workspace — bytes of device workspace moe_forward needs for these
+ * sizes (0 for invalid sizes).  The workspace holds the dispatch tables, the
+ * expert-sorted copy of x, the SwiGLU intermediates and the per-slot partial
+ * outputs; its size grows as N*k*(D + d_moe) + N*d_sh + E*(D + d_moe).
+ */
+size_t moe_forward_workspace(int N, int D, int E, int d_moe, int d_sh, int k, int dtype);
+
+/*
+ * moe_forward — routed experts, weighted combine and shared expert.
+ * Defined by "GLM-4.5 MoE Forward", How it works: each routed expert is the
+ * bias-free SwiGLU E_i(x) = W_down,i (SiLU(W_gate,i x) (.) W_up,i x) and
+ * y_n = sum_{i in T(n)} w_{n,i} E_i(x_n) + E_sh(x_n), the shared expert (width
+ * d_sh) on the same input at scale 1.  Weight layouts as in the GLM-5 "Mixture
+ * of experts" code excerpt: gate_up_proj[i] is (2 d_moe, D) with the gate rows
+ * first, down_proj[i] is (D, d_moe); an id equal to E is a sentinel that
+ * contributes nothing.  topk_w already holds alpha; nothing is renormalised.
+ *
+ *   x        [N, D]            dtype
+ *   gate_up  [E, 2*d_moe, D]   dtype
+ *   down     [E, D, d_moe]     dtype
+ *   sh_gate  [d_sh, D]         dtype
+ *   sh_up    [d_sh, D]         dtype
+ *   sh_down  [D, d_sh]         dtype
+ *   topk_idx [N, k]            int32, each in [0, E]
+ *   topk_w   [N, k]            fp32
+ *   y        [N, D]            dtype out, fully overwritten
+ *   workspace, ws_bytes        device scratch of at least moe_forward_workspace()
+ * dtype MOE_BF16 runs the tensor-core path (bf16 operands, fp32 accumulation,
+ * bf16 SwiGLU intermediate and per-slot partials, fp32 sum, one rounding of y);
+ * MOE_F32 runs an fp32 CUDA-core path.  N = 0 is a no-op.
+ * Ids outside [0, E] are skipped and reported by moe_device_status().
+ */
+int moe_forward(const void *x, const void *gate_up, const void *down, const void *sh_gate,
+                const void *sh_up, const void *sh_down, const int32_t *topk_idx,
+                const float *topk_w, int N, int D, int E, int d_moe, int d_sh, int k,
+                int dtype, void *y, void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * moe_device_status — synchronises `stream`, then returns and clears the device
+ * status word: MOE_OK, MOE_ERR_DEVICE_TIMEOUT (a bounded wait ran out; the
+ * output of that call is not valid) or MOE_ERR_BAD_INDEX.  Returns
+ * MOE_ERR_CUDA if the synchronisation itself failed.
+ */
+int moe_device_status(void *stream);
+
+/* Static, human-readable text for a status code. */
+const char *moe_status_string(int status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int moe_version(void);
+
+/*
+ * Test hooks for the bounded device-side waits (no GPU fault is involved).
+ *   moe_debug_set_wait_limit_ns: limit for every spin-wait in the kernels
+ *     (default 2e9 ns); ns = 0 restores the default.
+ *   moe_debug_never_signal: when on, the shared-expert combine of the next
+ *     moe_forward calls waits for one more routed tile than exists, so the wait
+ *     runs out, the status word reports MOE_ERR_DEVICE_TIMEOUT and the kernel
+ *     returns normally.
+ */
+int moe_debug_set_wait_limit_ns(uint64_t ns);
+int moe_debug_never_signal(int on);
+
+/*
+ * Profiling hooks (used by the benchmark; no effect on results).
+ *   moe_profile_set_events: while n > 0, every moe_forward call records
+ *     events[0] on its stream before its first kernel and events[i] right after
+ *     its i-th kernel launch (i = 1 .. n-1).  The events are caller-owned
+ *     cudaEvent_t handles passed as void*; n = 0 turns recording off.  At most
+ *     16 events; MOE_ERR_ARG otherwise.
+ *   moe_launch_count: kernels launched by this library in this process so far.
+ */
+int moe_profile_set_events(void *const *events, int n);
+unsigned long long moe_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

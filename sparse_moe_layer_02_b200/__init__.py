@@ -1,0 +1,210 @@
+"""B200 (sm_100a) sparse MoE FFN forward, GLM-4.5 / GLM-5 style.
+
+Thin ctypes binding over libmoe.so (C ABI in include/moe.h).  The functions
+here only marshal torch CUDA tensors into pointers, sizes and the current
+stream; every step of the layer runs in the library's CUDA kernels.  There is
+no fallback: if libmoe.so is missing or no sm_100 GPU is current, calls raise.
+
+    idx, w = moe_router(x, W_g, b, n_group, topk_group, k, norm_topk_prob, alpha)
+    y = moe_forward(x, gate_up, down, sh_gate, sh_up, sh_down, idx, w)
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+__all__ = ["MoEError", "moe_router", "moe_forward", "moe_forward_workspace", "moe_layer",
+           "moe_device_status", "moe_status_string", "moe_debug_set_wait_limit_ns",
+           "moe_debug_never_signal", "moe_profile_set_events", "moe_launch_count", "library_path", "load_library", "MOE_F32", "MOE_BF16",
+           "EXPORTED_SYMBOLS"]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libmoe.so")
+_lock = threading.Lock()
+_lib = None
+
+MOE_F32, MOE_BF16 = 0, 1
+MOE_OK = 0
+
+EXPORTED_SYMBOLS = ("moe_router", "moe_forward_workspace", "moe_forward", "moe_device_status",
+                    "moe_status_string", "moe_version", "moe_debug_set_wait_limit_ns",
+                    "moe_debug_never_signal", "moe_profile_set_events", "moe_launch_count")
+
+
+class MoEError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__("%s failed: %s (status %d)" % (what, moe_status_string(code), code))
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load_library():
+    """Load libmoe.so (built in-tree by sparse_moe_layer_02_b200.build); raise if absent."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError("libmoe.so not found at %s; build it with "
+                               "`python -m sparse_moe_layer_02_b200.build`" % _LIB_PATH)
+        lib = ctypes.CDLL(_LIB_PATH)
+        P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+        lib.moe_router.argtypes = [P, I, P, I, P, I, I, I, I, I, I, I, F, P, P, P]
+        lib.moe_router.restype = I
+        lib.moe_forward_workspace.argtypes = [I, I, I, I, I, I, I]
+        lib.moe_forward_workspace.restype = ctypes.c_size_t
+        lib.moe_forward.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, P, P,
+                                    ctypes.c_size_t, P]
+        lib.moe_forward.restype = I
+        lib.moe_device_status.argtypes = [P]
+        lib.moe_device_status.restype = I
+        lib.moe_status_string.argtypes = [I]
+        lib.moe_status_string.restype = ctypes.c_char_p
+        lib.moe_version.argtypes = []
+        lib.moe_version.restype = I
+        lib.moe_debug_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+        lib.moe_debug_set_wait_limit_ns.restype = I
+        lib.moe_debug_never_signal.argtypes = [I]
+        lib.moe_debug_never_signal.restype = I
+        lib.moe_profile_set_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), I]
+        lib.moe_profile_set_events.restype = I
+        lib.moe_launch_count.argtypes = []
+        lib.moe_launch_count.restype = ctypes.c_ulonglong
+        _lib = lib
+        return lib
+
+
+def moe_status_string(code: int) -> str:
+    return load_library().moe_status_string(int(code)).decode()
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return MOE_F32
+    if t.dtype == torch.bfloat16:
+        return MOE_BF16
+    raise TypeError("unsupported dtype %s (float32 or bfloat16)" % t.dtype)
+
+
+def _dev(t: torch.Tensor, name: str) -> int:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor" % name)
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    return t.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _check(rc: int, what: str):
+    if rc != MOE_OK:
+        raise MoEError(rc, what)
+
+
+def moe_router(x, W_g, b, n_group: int, topk_group: int, k: int, norm_topk_prob: bool,
+               alpha: float, topk_idx=None, topk_w=None, stream=None):
+    """Router: returns (topk_idx [N,k] int32, topk_w [N,k] fp32) on x's device."""
+    lib = load_library()
+    N, D = x.shape
+    E = W_g.shape[0]
+    if tuple(W_g.shape) != (E, D) or tuple(b.shape) != (E,) or b.dtype != torch.float32:
+        raise ValueError("W_g must be [E, D] and b [E] float32")
+    if topk_idx is None:
+        topk_idx = torch.empty((N, k), dtype=torch.int32, device=x.device)
+    if topk_w is None:
+        topk_w = torch.empty((N, k), dtype=torch.float32, device=x.device)
+    if topk_idx.dtype != torch.int32 or topk_w.dtype != torch.float32:
+        raise ValueError("topk_idx must be int32 and topk_w float32")
+    if tuple(topk_idx.shape) != (N, k) or tuple(topk_w.shape) != (N, k):
+        raise ValueError("topk_idx / topk_w must be [N, k]")
+    rc = lib.moe_router(_dev(x, "x"), _dt(x), _dev(W_g, "W_g"), _dt(W_g), _dev(b, "b"), N, D, E,
+                        int(n_group), int(topk_group), int(k), int(bool(norm_topk_prob)),
+                        float(alpha), _dev(topk_idx, "topk_idx"), _dev(topk_w, "topk_w"),
+                        _stream(stream))
+    _check(rc, "moe_router")
+    return topk_idx, topk_w
+
+
+def moe_forward_workspace(N: int, D: int, E: int, d_moe: int, d_sh: int, k: int,
+                          dtype: torch.dtype) -> int:
+    return int(load_library().moe_forward_workspace(N, D, E, d_moe, d_sh, k,
+                                                     MOE_BF16 if dtype == torch.bfloat16 else MOE_F32))
+
+
+def moe_forward(x, gate_up, down, sh_gate, sh_up, sh_down, topk_idx, topk_w, y=None,
+                workspace=None, stream=None):
+    """Routed experts + weighted combine + shared expert; returns y [N, D]."""
+    lib = load_library()
+    N, D = x.shape
+    E, two_d, D2 = gate_up.shape
+    d = two_d // 2
+    d_sh = sh_gate.shape[0]
+    k = topk_idx.shape[1] if topk_idx.dim() == 2 else 0
+    if D2 != D or tuple(down.shape) != (E, D, d) or tuple(sh_up.shape) != (d_sh, D) \
+            or tuple(sh_down.shape) != (D, d_sh) or tuple(topk_w.shape) != (N, k):
+        raise ValueError("inconsistent expert or routing shapes")
+    for t in (gate_up, down, sh_gate, sh_up, sh_down):
+        if t.dtype != x.dtype:
+            raise ValueError("expert weights must share x's dtype")
+    if topk_idx.dtype != torch.int32 or topk_w.dtype != torch.float32:
+        raise ValueError("topk_idx must be int32 and topk_w float32")
+    if y is None:
+        y = torch.empty((N, D), dtype=x.dtype, device=x.device)
+    ws_bytes = int(lib.moe_forward_workspace(N, D, E, d, d_sh, k, _dt(x)))
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=x.device)
+    rc = lib.moe_forward(_dev(x, "x"), _dev(gate_up, "gate_up"), _dev(down, "down"),
+                         _dev(sh_gate, "sh_gate"), _dev(sh_up, "sh_up"), _dev(sh_down, "sh_down"),
+                         _dev(topk_idx, "topk_idx"), _dev(topk_w, "topk_w"), N, D, E, d, d_sh, k,
+                         _dt(x), _dev(y, "y"), _dev(workspace, "workspace"),
+                         workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc, "moe_forward")
+    return y
+
+
+def moe_layer(x, W_g, b, gate_up, down, sh_gate, sh_up, sh_down, n_group, topk_group, k,
+              norm_topk_prob, alpha, workspace=None, y=None, topk_idx=None, topk_w=None,
+              stream=None):
+    """Whole layer: router then forward.  Returns (y, topk_idx, topk_w)."""
+    idx, w = moe_router(x, W_g, b, n_group, topk_group, k, norm_topk_prob, alpha, topk_idx,
+                        topk_w, stream)
+    y = moe_forward(x, gate_up, down, sh_gate, sh_up, sh_down, idx, w, y, workspace, stream)
+    return y, idx, w
+
+
+def moe_device_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device status word."""
+    return int(load_library().moe_device_status(_stream(stream)))
+
+
+def moe_debug_set_wait_limit_ns(ns: int):
+    _check(load_library().moe_debug_set_wait_limit_ns(int(ns)), "moe_debug_set_wait_limit_ns")
+
+
+def moe_debug_never_signal(on: bool):
+    _check(load_library().moe_debug_never_signal(int(bool(on))), "moe_debug_never_signal")
+
+
+def moe_profile_set_events(events) -> None:
+    """Record the given torch.cuda.Event objects at moe_forward's kernel boundaries
+    (events[0] before the first kernel, events[i] after the i-th); [] turns it off."""
+    handles = [int(e.cuda_event) for e in events]
+    arr = (ctypes.c_void_p * max(len(handles), 1))(*handles)
+    _check(load_library().moe_profile_set_events(arr, len(handles)), "moe_profile_set_events")
+
+
+def moe_launch_count() -> int:
+    return int(load_library().moe_launch_count())

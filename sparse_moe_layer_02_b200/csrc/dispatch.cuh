@@ -1,0 +1,188 @@
+// Token dispatch ("GLM-4.5 MoE Forward", How it works: token-choice dispatch,
+// every token goes to exactly its k routed experts; an id equal to E is the
+// sentinel of the GLM-5 experts' forward and goes nowhere).
+//
+// The N*k (token, slot) pairs are sorted by (expert, token, slot) into
+// expert-contiguous segments, each padded to a multiple of 128 rows so every
+// 128-row tile of the permuted layout belongs to one expert:
+//   1. count:   per-chunk expert histograms (shared-memory atomics)
+//   2. scan:    per-expert totals, per-chunk bases, 128-row tile prefix
+//   3. scatter: stable positions (warp match + per-warp counts), inverse map,
+//               per-row token id and routing weight
+//   4. gather:  copy each token's row of x to its permuted rows (bf16 path)
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int DISPATCH_CHUNK = 1024;
+constexpr int DISPATCH_THREADS = 256;
+constexpr int DISPATCH_MAXE = 512;
+constexpr int TILE_M = 128;
+
+struct DispatchParams {
+    const int32_t *topk_idx; // [N*k]
+    const float *topk_w;     // [N*k]
+    int N, k, E, nchunks;
+    int32_t *chunk_hist; // [nchunks][E] counts, then absolute bases
+    int32_t *counts;     // [E]
+    int32_t *tile_off;   // [E+1] prefix of 128-row tiles per expert
+    int32_t *meta;       // [0] done counter, [1] padded rows, [2] routed m-tiles
+    int32_t *pos_of;     // [N*k] permuted row of each (token, slot), -1 if none
+    int32_t *perm_tok;   // [rows_max] token of each permuted row, -1 for padding
+    float *w_perm;       // [rows_max] routing weight of each permuted row, 0 for padding
+};
+
+__global__ void __launch_bounds__(DISPATCH_THREADS) dispatch_count_kernel(const DispatchParams p) {
+    __shared__ int hist[DISPATCH_MAXE];
+    for (int e = threadIdx.x; e < p.E; e += blockDim.x) hist[e] = 0;
+    __syncthreads();
+    const int total = p.N * p.k;
+    const int base = blockIdx.x * DISPATCH_CHUNK;
+    for (int i = base + threadIdx.x; i < min(base + DISPATCH_CHUNK, total); i += blockDim.x) {
+        const int e = p.topk_idx[i];
+        if (e >= 0 && e < p.E)
+            atomicAdd(&hist[e], 1);
+        else if (e != p.E)
+            record_error(DEV_BAD_INDEX, 10);
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < p.E; e += blockDim.x)
+        p.chunk_hist[(size_t)blockIdx.x * p.E + e] = hist[e];
+}
+
+// One CTA of DISPATCH_MAXE threads (thread e owns expert e).
+__global__ void __launch_bounds__(DISPATCH_MAXE) dispatch_scan_kernel(const DispatchParams p) {
+    __shared__ int wsum[DISPATCH_MAXE / 32];
+    const int e = threadIdx.x;
+    const int lane = e & 31, warp = e >> 5;
+    int total = 0;
+    if (e < p.E) {
+        for (int c = 0; c < p.nchunks; ++c) {
+            int *h = &p.chunk_hist[(size_t)c * p.E + e];
+            const int v = *h;
+            *h = total; // exclusive within the expert
+            total += v;
+        }
+        p.counts[e] = total;
+    }
+    const int tiles = (e < p.E) ? (total + TILE_M - 1) / TILE_M : 0;
+    // Block-wide exclusive scan of tiles.
+    int v = tiles;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, v, off);
+        if (lane >= off) v += n;
+    }
+    if (lane == 31) wsum[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+        int w = (lane < DISPATCH_MAXE / 32) ? wsum[lane] : 0;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int n = __shfl_up_sync(0xffffffffu, w, off);
+            if (lane >= off) w += n;
+        }
+        if (lane < DISPATCH_MAXE / 32) wsum[lane] = w;
+    }
+    __syncthreads();
+    const int incl = v + (warp > 0 ? wsum[warp - 1] : 0);
+    const int excl = incl - tiles;
+    if (e < p.E) {
+        p.tile_off[e] = excl;
+        const int row0 = excl * TILE_M;
+        for (int c = 0; c < p.nchunks; ++c) p.chunk_hist[(size_t)c * p.E + e] += row0;
+        for (int r = row0 + total; r < row0 + tiles * TILE_M; ++r) {
+            p.perm_tok[r] = -1;
+            p.w_perm[r] = 0.f;
+        }
+    }
+    if (e == p.E - 1) {
+        p.tile_off[p.E] = incl;
+        p.meta[0] = 0;
+        p.meta[1] = incl * TILE_M;
+        p.meta[2] = incl;
+    }
+}
+
+__global__ void __launch_bounds__(DISPATCH_THREADS) dispatch_scatter_kernel(const DispatchParams p) {
+    constexpr int NW = DISPATCH_THREADS / 32;
+    __shared__ int cursor[DISPATCH_MAXE];
+    __shared__ int wcnt[NW][DISPATCH_MAXE];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    for (int e = tid; e < p.E; e += DISPATCH_THREADS) {
+        cursor[e] = p.chunk_hist[(size_t)blockIdx.x * p.E + e];
+#pragma unroll
+        for (int w = 0; w < NW; ++w) wcnt[w][e] = 0;
+    }
+    __syncthreads();
+    const int total = p.N * p.k;
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    for (int round = 0; round < DISPATCH_CHUNK / DISPATCH_THREADS; ++round) {
+        const int i = blockIdx.x * DISPATCH_CHUNK + round * DISPATCH_THREADS + tid;
+        const bool valid = i < total;
+        int key = -1;
+        if (valid) {
+            const int e = p.topk_idx[i];
+            key = (e >= 0 && e < p.E) ? e : -1;
+        }
+        const uint32_t peers = __match_any_sync(0xffffffffu, key);
+        const int rank = __popc(peers & lt_mask);
+        if (key >= 0 && rank == 0) wcnt[warp][key] = __popc(peers);
+        __syncthreads();
+        int pos = -1;
+        if (key >= 0) {
+            pos = cursor[key] + rank;
+            for (int w = 0; w < warp; ++w) pos += wcnt[w][key];
+        }
+        __syncthreads();
+        for (int e = tid; e < p.E; e += DISPATCH_THREADS) {
+            int add = 0;
+#pragma unroll
+            for (int w = 0; w < NW; ++w) {
+                add += wcnt[w][e];
+                wcnt[w][e] = 0;
+            }
+            cursor[e] += add;
+        }
+        if (valid) {
+            p.pos_of[i] = pos;
+            if (pos >= 0) {
+                p.perm_tok[pos] = i / p.k;
+                p.w_perm[pos] = p.topk_w[i];
+            }
+        }
+        __syncthreads();
+    }
+}
+
+// Copy x[perm_tok[r]] to x_perm[r] for every real permuted row; one warp per row,
+// 16-byte vectors.  row_bytes is a multiple of 16.
+__global__ void __launch_bounds__(256) dispatch_gather_kernel(const uint8_t *__restrict__ x,
+                                                              uint8_t *__restrict__ x_perm,
+                                                              const int32_t *perm_tok,
+                                                              const int32_t *meta,
+                                                              int row_bytes, int rows_max) {
+    const int rows = min(meta[1], rows_max);
+    const int lane = threadIdx.x & 31;
+    for (int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < rows;
+         r += (gridDim.x * blockDim.x) >> 5) {
+        const int tok = perm_tok[r];
+        if (tok < 0) continue;
+        const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)tok * row_bytes);
+        uint4 *dst = reinterpret_cast<uint4 *>(x_perm + (size_t)r * row_bytes);
+        const int nvec = row_bytes >> 4;
+        int v = lane;
+        for (; v + 96 < nvec; v += 128) {
+            const uint4 a = src[v], b = src[v + 32], c = src[v + 64], d = src[v + 96];
+            dst[v] = a;
+            dst[v + 32] = b;
+            dst[v + 64] = c;
+            dst[v + 96] = d;
+        }
+        for (; v < nvec; v += 32) dst[v] = src[v];
+    }
+}
+
+}  // namespace moe

@@ -1,0 +1,395 @@
+// Grouped expert GEMMs on the 5th-generation tensor cores (tcgen05 + TMEM + TMA).
+//
+// Both kernels are persistent (one CTA per SM, static round-robin over tiles) and
+// warp-specialised, 192 threads:
+//   warp 0      TMA producer: A tile 128 x 64 and B tile 256 x 64 (bf16, 128-byte
+//               swizzle) per stage into a 4-stage shared-memory ring
+//   warp 1      allocates 512 TMEM columns and issues tcgen05.mma (M=128, N=256,
+//               K=16, bf16 in, fp32 accumulate) from one thread; two 256-column
+//               accumulators alternate so the epilogue of one tile overlaps the
+//               main loop of the next
+//   warps 2-5   epilogue: tcgen05.ld of the accumulator (warp w reads TMEM lanes
+//               32*(w%4) .. +31, i.e. one output row per thread), math, stores
+//
+// gate_up ("GLM-4.5 MoE Forward": E_i(x) = W_down (SiLU(W_gate x) (.) W_up x);
+// gate_up_proj[i] is (2 d_moe, D), gate rows first): one tile = 128 permuted
+// token rows x 128 intermediate columns; B stacks 128 gate rows and the matching
+// 128 up rows, so accumulator columns 0..127 hold the gate and 128..255 the up
+// projection of the same columns and the epilogue writes h = SiLU(gate) * up in
+// bf16.  The shared expert's tiles (A = x itself, B = its gate/up matrices) follow
+// the routed tiles in the same launch.
+//
+// down: one tile = 128 rows x 256 output columns of W_down (D x d_moe).  Routed
+// tiles scale each row by its routing weight and store a bf16 per-slot partial.
+// The shared expert's tiles come last: after a bounded wait until every routed
+// tile is stored, each row n adds its k slot partials in slot order and the
+// shared expert's fp32 accumulator (scale 1), and writes y once in bf16
+// (deterministic: no atomics on the output).
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int GEMM_BM = 128;
+constexpr int GEMM_BN = 256;
+constexpr int GEMM_BK = 64;
+constexpr int GEMM_STAGES = 4;
+constexpr int GEMM_THREADS = 192;
+constexpr int GEMM_A_BYTES = GEMM_BM * GEMM_BK * 2;  // 16 KiB
+constexpr int GEMM_B_BYTES = GEMM_BN * GEMM_BK * 2;  // 32 KiB
+constexpr int GEMM_STAGE_BYTES = GEMM_A_BYTES + GEMM_B_BYTES;
+constexpr int GEMM_TMEM_COLS = 512;
+constexpr int GEMM_MAXE = 512;
+// Shared memory: 1024 alignment slack + ring + barriers/flags + tile table.
+constexpr int GEMM_SMEM_BYTES =
+    1024 + GEMM_STAGES * GEMM_STAGE_BYTES + 256 + (GEMM_MAXE + 1) * 4 + 64;
+
+enum GemmKind { GEMM_GATE_UP = 0, GEMM_DOWN = 1 };
+
+struct GemmArgs {
+    const int32_t *tile_off; // [E+1]
+    int32_t *meta;           // [0] routed tiles done (down), [2] routed m-tiles
+    int E, N, k;
+    int nb_r, nb_s;      // n-blocks per routed / shared m-tile
+    int mt_s;            // shared m-tiles
+    int kb_r, kb_s;      // k-blocks of routed / shared tiles
+    int b_rows_per_e;    // rows of one expert in the routed B map (2d or D)
+    int up_off;          // gate_up: row offset of the up half (d)
+    // outputs
+    __nv_bfloat16 *out_r; // gate_up: h_perm [rows, ld_r]; down: slot [rows, ld_r]
+    int ld_r, ncols_r;
+    __nv_bfloat16 *out_s; // gate_up: h_sh [N, ld_s]; down: y [N, ld_s]
+    int ld_s, ncols_s;
+    const float *w_perm;   // down: routing weight per permuted row
+    const int32_t *pos_of; // down: [N*k] permuted row of (n, j), -1 if none
+    const __nv_bfloat16 *slot; // down: slot partials (same as out_r)
+    uint64_t wait_limit_ns;
+    int never_signal;
+};
+
+struct TileCoord {
+    bool shared;
+    int e;     // routed expert
+    int a_row; // row coordinate in the A map
+    int nb;    // n-block
+    int kb;    // k-blocks
+};
+
+__device__ __forceinline__ TileCoord decode_tile(int t, int routed_tiles, const GemmArgs &a,
+                                                 const int *s_tile_off) {
+    TileCoord c;
+    if (t < routed_tiles) {
+        const int mt = t / a.nb_r;
+        c.nb = t - mt * a.nb_r;
+        int lo = 0, hi = a.E - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (s_tile_off[mid] <= mt) lo = mid; else hi = mid - 1;
+        }
+        c.shared = false;
+        c.e = lo;
+        c.a_row = mt * GEMM_BM;
+        c.kb = a.kb_r;
+    } else {
+        const int t2 = t - routed_tiles;
+        const int mt = t2 / a.nb_s;
+        c.nb = t2 - mt * a.nb_s;
+        c.shared = true;
+        c.e = -1;
+        c.a_row = mt * GEMM_BM;
+        c.kb = a.kb_s;
+    }
+    return c;
+}
+
+__device__ __forceinline__ int ld_acquire_gpu(const int *p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Store 32 consecutive fp32 values as bf16 (cols [col, col+32) of a row), only the
+// 8-column pieces that lie below ncols (ncols % 8 == 0).
+__device__ __forceinline__ void store_row_chunk_bf16(__nv_bfloat16 *row_ptr, int col, int ncols,
+                                                     const float (&v)[32]) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+    uint4 *dst = reinterpret_cast<uint4 *>(row_ptr + col);
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+        if (col + 8 * q < ncols) dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+}
+
+template <int KIND>
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap mA_r,
+                        const __grid_constant__ CUtensorMap mB_r,
+                        const __grid_constant__ CUtensorMap mA_s,
+                        const __grid_constant__ CUtensorMap mB_s0,
+                        const __grid_constant__ CUtensorMap mB_s1, const GemmArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint8_t *ring = smem;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + GEMM_STAGES * GEMM_STAGE_BYTES);
+    uint64_t *empty = full + GEMM_STAGES;
+    uint64_t *tfull = empty + GEMM_STAGES;
+    uint64_t *tempty = tfull + 2;
+    uint64_t *drain = tempty + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    volatile int *combine_failed = abort_flag + 1;
+    int *s_tile_off = reinterpret_cast<int *>(smem + GEMM_STAGES * GEMM_STAGE_BYTES + 256);
+
+    const int warp = warp_id(), lane = lane_id();
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < GEMM_STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&tfull[i], 1);
+            mbar_init(&tempty[i], 4);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        *combine_failed = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&mA_r);
+        tma_prefetch_desc(&mB_r);
+        tma_prefetch_desc(&mA_s);
+        tma_prefetch_desc(&mB_s0);
+        if (KIND == GEMM_GATE_UP) tma_prefetch_desc(&mB_s1);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, GEMM_TMEM_COLS);
+        tmem_relinquish();
+    }
+    for (int i = threadIdx.x; i <= a.E; i += blockDim.x) s_tile_off[i] = a.tile_off[i];
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const int routed_tiles = a.meta[2] * a.nb_r;
+    const int total_tiles = routed_tiles + a.mt_s * a.nb_s;
+    const uint64_t limit = a.wait_limit_ns;
+
+    if (warp == 0) {
+        // ------------------------------ TMA producer ------------------------------
+        if (lane == 0) {
+            uint32_t it = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+                const TileCoord c = decode_tile(t, routed_tiles, a, s_tile_off);
+                const CUtensorMap *mA = c.shared ? &mA_s : &mA_r;
+                for (int kb = 0; kb < c.kb; ++kb, ++it) {
+                    const uint32_t s = it % GEMM_STAGES, ph = (it / GEMM_STAGES) & 1;
+                    if (!mbar_wait(&empty[s], ph ^ 1, limit, abort_flag, 100)) { ok = false; break; }
+                    uint8_t *sa = ring + s * GEMM_STAGE_BYTES;
+                    uint8_t *sb = sa + GEMM_A_BYTES;
+                    mbar_arrive_expect_tx(&full[s], GEMM_STAGE_BYTES);
+                    const int kx = kb * GEMM_BK;
+                    tma_load_2d(mA, &full[s], sa, kx, c.a_row);
+                    if (KIND == GEMM_GATE_UP) {
+                        if (c.shared) {
+                            tma_load_2d(&mB_s0, &full[s], sb, kx, c.nb * 128);
+                            tma_load_2d(&mB_s1, &full[s], sb + GEMM_B_BYTES / 2, kx, c.nb * 128);
+                        } else {
+                            const int r0 = c.e * a.b_rows_per_e + c.nb * 128;
+                            tma_load_2d(&mB_r, &full[s], sb, kx, r0);
+                            tma_load_2d(&mB_r, &full[s], sb + GEMM_B_BYTES / 2, kx, r0 + a.up_off);
+                        }
+                    } else {
+                        if (c.shared)
+                            tma_load_2d(&mB_s0, &full[s], sb, kx, c.nb * GEMM_BN);
+                        else
+                            tma_load_2d(&mB_r, &full[s], sb, kx, c.e * a.b_rows_per_e + c.nb * GEMM_BN);
+                    }
+                }
+            }
+            if (!ok) {
+                // Let copies already issued land before the CTA's memory goes away.
+                const uint32_t first = it > GEMM_STAGES ? it - GEMM_STAGES : 0;
+                for (uint32_t j = first; j < it; ++j) {
+                    volatile int no_abort = 0;
+                    mbar_wait(&full[j % GEMM_STAGES], (j / GEMM_STAGES) & 1, 10000000ull, &no_abort, 101);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------ MMA issuer --------------------------------
+        if (lane == 0) {
+            constexpr uint32_t idesc = umma_idesc_bf16(GEMM_BM, GEMM_BN);
+            uint32_t it = 0, tc = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++tc) {
+                const TileCoord c = decode_tile(t, routed_tiles, a, s_tile_off);
+                const uint32_t acc = tc & 1, aph = (tc >> 1) & 1;
+                if (!mbar_wait(&tempty[acc], aph ^ 1, limit, abort_flag, 110)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + acc * GEMM_BN;
+                for (int kb = 0; kb < c.kb; ++kb, ++it) {
+                    const uint32_t s = it % GEMM_STAGES, ph = (it / GEMM_STAGES) & 1;
+                    if (!mbar_wait(&full[s], ph, limit, abort_flag, 111)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t sa = smem_u32(ring + s * GEMM_STAGE_BYTES);
+                    const uint32_t sb = sa + GEMM_A_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < GEMM_BK / 16; ++kk)
+                        umma_bf16_ss(d_tmem, umma_desc_sw128(sa + kk * 32),
+                                     umma_desc_sw128(sb + kk * 32), idesc,
+                                     (kb > 0 || kk > 0) ? 1u : 0u);
+                    umma_commit(&empty[s]);
+                }
+                if (!ok) break;
+                umma_commit(&tfull[acc]);
+            }
+            // Drain: wait until every MMA issued by this thread has completed.
+            umma_commit(drain);
+            volatile int no_abort = 0;
+            mbar_wait(drain, 0, 100000000ull, &no_abort, 112);
+        }
+    } else {
+        // ------------------------------ epilogue ---------------------------------
+        const int q = warp & 3;          // TMEM lane quadrant of this warp
+        const int row = q * 32 + lane;   // row of the tile owned by this thread
+        const int ep_tid = threadIdx.x - 64;
+        uint32_t tc = 0;
+        for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++tc) {
+            const TileCoord c = decode_tile(t, routed_tiles, a, s_tile_off);
+            const uint32_t acc = tc & 1, aph = (tc >> 1) & 1;
+            bool do_combine = true;
+            if (KIND == GEMM_DOWN && c.shared) {
+                // Wait until every routed tile has stored its slot partials.
+                if (ep_tid == 0 && !*combine_failed && !*abort_flag) {
+                    const int target = routed_tiles + (a.never_signal ? 1 : 0);
+                    const uint64_t t0 = globaltimer_ns();
+                    while (ld_acquire_gpu(&a.meta[0]) < target) {
+                        if (globaltimer_ns() - t0 > limit) {
+                            record_error(DEV_TIMEOUT, 120);
+                            *combine_failed = 1;
+                            break;
+                        }
+                        __nanosleep(200);
+                    }
+                }
+                named_bar_sync(1, 128);
+                do_combine = !*combine_failed;
+            }
+            // After an abort every wait fails at once; the loop still walks the same
+            // tiles in every epilogue warp so the named barriers stay matched.
+            // One lane waits; the result is made warp-uniform before the
+            // warp-collective TMEM loads.
+            bool have = false;
+            if (lane == 0) have = mbar_wait(&tfull[acc], aph, limit, abort_flag, 121);
+            have = __shfl_sync(0xffffffffu, have ? 1 : 0, 0) != 0;
+            __syncwarp();
+            if (have) {
+            tc_fence_after();
+            const uint32_t tbase = tmem_base + acc * GEMM_BN + ((uint32_t)(q * 32) << 16);
+
+            if (KIND == GEMM_GATE_UP) {
+                __nv_bfloat16 *out = c.shared ? a.out_s : a.out_r;
+                const int ld = c.shared ? a.ld_s : a.ld_r;
+                const int ncols = c.shared ? a.ncols_s : a.ncols_r;
+                const int grow = c.a_row + row;
+                const bool row_ok = c.shared ? (grow < a.N) : true;
+                __nv_bfloat16 *row_ptr = out + (size_t)grow * ld;
+#pragma unroll 1
+                for (int ch = 0; ch < 4; ++ch) {
+                    uint32_t g[32], u[32];
+                    tmem_ld_32x32b_x32(tbase + ch * 32, g);
+                    tmem_ld_32x32b_x32(tbase + 128 + ch * 32, u);
+                    tmem_ld_wait();
+                    const int col = c.nb * 128 + ch * 32;
+                    if (row_ok && col < ncols) {
+                        float h[32];
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            h[i] = silu_f(__uint_as_float(g[i])) * __uint_as_float(u[i]);
+                        store_row_chunk_bf16(row_ptr, col, ncols, h);
+                    }
+                }
+            } else if (!c.shared) {
+                const int grow = c.a_row + row;
+                const float wr = a.w_perm[grow];
+                __nv_bfloat16 *row_ptr = a.out_r + (size_t)grow * a.ld_r;
+#pragma unroll 1
+                for (int ch = 0; ch < 8; ++ch) {
+                    uint32_t v[32];
+                    tmem_ld_32x32b_x32(tbase + ch * 32, v);
+                    tmem_ld_wait();
+                    const int col = c.nb * GEMM_BN + ch * 32;
+                    if (col < a.ncols_r) {
+                        float o[32];
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) o[i] = wr * __uint_as_float(v[i]);
+                        store_row_chunk_bf16(row_ptr, col, a.ncols_r, o);
+                    }
+                }
+            } else {
+                const int n = c.a_row + row;
+                const bool row_ok = n < a.N && do_combine;
+                __nv_bfloat16 *row_ptr = a.out_s + (size_t)n * a.ld_s;
+#pragma unroll 1
+                for (int ch = 0; ch < 8; ++ch) {
+                    uint32_t v[32];
+                    tmem_ld_32x32b_x32(tbase + ch * 32, v);
+                    tmem_ld_wait();
+                    const int col = c.nb * GEMM_BN + ch * 32;
+                    if (row_ok && col < a.ncols_s) {
+                        float sum[32];
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) sum[i] = 0.f;
+                        for (int j = 0; j < a.k; ++j) {
+                            const int p = a.pos_of[(size_t)n * a.k + j];
+                            if (p < 0) continue;
+                            const uint4 *src =
+                                reinterpret_cast<const uint4 *>(a.slot + (size_t)p * a.ld_r + col);
+#pragma unroll
+                            for (int qv = 0; qv < 4; ++qv) {
+                                if (col + 8 * qv < a.ncols_s) {
+                                    const uint4 w4 = __ldcg(src + qv);
+                                    float lo, hi;
+                                    unpack_bf16x2(w4.x, lo, hi); sum[8 * qv + 0] += lo; sum[8 * qv + 1] += hi;
+                                    unpack_bf16x2(w4.y, lo, hi); sum[8 * qv + 2] += lo; sum[8 * qv + 3] += hi;
+                                    unpack_bf16x2(w4.z, lo, hi); sum[8 * qv + 4] += lo; sum[8 * qv + 5] += hi;
+                                    unpack_bf16x2(w4.w, lo, hi); sum[8 * qv + 6] += lo; sum[8 * qv + 7] += hi;
+                                }
+                            }
+                        }
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) sum[i] += __uint_as_float(v[i]);
+                        store_row_chunk_bf16(row_ptr, col, a.ncols_s, sum);
+                    }
+                }
+            }
+            // Release the accumulator.
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[acc]);
+            }  // have
+            if (KIND == GEMM_DOWN && !c.shared) {
+                // Publish this routed tile's partials to the shared-expert tiles.
+                __threadfence();
+                named_bar_sync(1, 128);
+                if (ep_tid == 0 && have) atomicAdd(&a.meta[0], 1);
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, GEMM_TMEM_COLS);
+    }
+}
+
+}  // namespace moe

@@ -1,0 +1,490 @@
+// C-ABI entry points of libmoe: argument checks, workspace planning, TMA
+// descriptor encoding and kernel launches.  Declarations and the contract of
+// every entry point are in include/moe.h.
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "../../include/moe.h"
+#include "common.cuh"
+#include "dispatch.cuh"
+#include "gemm_sm100.cuh"
+#include "router.cuh"
+#include "simt_f32.cuh"
+
+namespace moe {
+namespace {
+
+constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;
+uint64_t g_wait_limit_ns = kDefaultWaitLimitNs;
+int g_never_signal = 0;
+
+std::atomic<unsigned long long> g_launches{0};
+constexpr int kMaxProfEvents = 16;
+void *g_prof_events[kMaxProfEvents];
+int g_prof_n = 0;
+
+// Records the caller's profiling events (if any) at kernel boundaries of one call.
+struct Profiler {
+    cudaStream_t st;
+    int next = 0;
+    explicit Profiler(cudaStream_t s) : st(s) { mark(); }
+    void mark() {
+        if (next < g_prof_n && g_prof_events[next])
+            cudaEventRecord(static_cast<cudaEvent_t>(g_prof_events[next]), st);
+        ++next;
+    }
+};
+
+constexpr int kMaxDevices = 64;
+struct DeviceInfo {
+    bool ready;
+    int sms;
+    int major, minor;
+    bool gemm_attr_set;
+    bool router_attr_set;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_mu;
+
+int current_device_info(DeviceInfo **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    DeviceInfo &d = g_dev[dev];
+    if (!d.ready) {
+        cudaDeviceProp prop;
+        if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return MOE_ERR_CUDA;
+        d.sms = prop.multiProcessorCount;
+        d.major = prop.major;
+        d.minor = prop.minor;
+        d.ready = true;
+    }
+    *out = &d;
+    return MOE_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+int check_router_shape(int N, int D, int E, int G, int tg, int k) {
+    if (N < 0 || N > 65535 * ROUTER_TM || D <= 0 || E <= 0 || E > DISPATCH_MAXE)
+        return MOE_ERR_SHAPE;
+    if (G <= 0 || G > ROUTER_MAXG || E % G != 0) return MOE_ERR_SHAPE;
+    if (G > 1 && E / G < 2) return MOE_ERR_SHAPE;
+    if (tg <= 0 || tg > G) return MOE_ERR_SHAPE;
+    if (k <= 0 || k > 32 || k > tg * (E / G)) return MOE_ERR_SHAPE;
+    return MOE_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Workspace layout (every region 256-byte aligned).
+// ---------------------------------------------------------------------------
+struct WsLayout {
+    size_t chunk_hist, counts, tile_off, meta, pos_of, perm_tok, w_perm;
+    size_t x_perm, h_perm, h_sh, slot, total;
+    int nchunks;
+    size_t rows_max;
+};
+
+bool plan_workspace(int N, int D, int E, int d, int d_sh, int k, int dtype, WsLayout &L) {
+    if (N < 0 || D <= 0 || E <= 0 || d <= 0 || d_sh <= 0 || k <= 0) return false;
+    if (dtype != MOE_F32 && dtype != MOE_BF16) return false;
+    const size_t es = dtype == MOE_BF16 ? 2 : 4;
+    const size_t nk = (size_t)N * (size_t)k;
+    if (nk > (size_t)INT32_MAX / 2) return false;
+    L.rows_max = round_up(nk + (size_t)(TILE_M - 1) * E, TILE_M);
+    if (L.rows_max > (size_t)INT32_MAX / 2) return false;
+    L.nchunks = (int)((nk + DISPATCH_CHUNK - 1) / DISPATCH_CHUNK);
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = off;
+        off = round_up(off + bytes, 256);
+        return at;
+    };
+    L.chunk_hist = take((size_t)std::max(L.nchunks, 1) * E * 4);
+    L.counts = take((size_t)E * 4);
+    L.tile_off = take((size_t)(E + 1) * 4);
+    L.meta = take(16 * 4);
+    L.pos_of = take(nk * 4);
+    L.perm_tok = take(L.rows_max * 4);
+    L.w_perm = take(L.rows_max * 4);
+    L.x_perm = take(dtype == MOE_BF16 ? L.rows_max * D * es : 0);
+    L.h_perm = take(L.rows_max * d * es);
+    L.h_sh = take((size_t)N * d_sh * es);
+    L.slot = take(L.rows_max * D * es);
+    L.total = off;
+    return true;
+}
+
+// ---------------------------------------------------------------------------
+// TMA descriptors
+// ---------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 2-D bf16 map over a row-major [rows, cols] matrix with row stride ld elements;
+// box = 64 columns (128 bytes, the swizzle span) x box_rows rows, 128-byte swizzle,
+// out-of-range elements read as zero.
+bool make_map(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows, uint64_t ld,
+              uint32_t box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {ld * 2};
+    cuuint32_t box[2] = {GEMM_BK, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+int launch_status() {
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int launched(Profiler &prof) {
+    const int rc = launch_status();
+    prof.mark();
+    return rc;
+}
+
+template <typename XT, typename WT, int TE>
+int launch_router_t(const RouterParams &p, cudaStream_t st) {
+    const int CL = (p.E + TE - 1) / TE;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(CL, (p.N + ROUTER_TM - 1) / ROUTER_TM, 1);
+    cfg.blockDim = dim3(ROUTER_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = CL;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, router_kernel<XT, WT, TE>, p) != cudaSuccess) return MOE_ERR_CUDA;
+    return launch_status();
+}
+
+template <typename XT, typename WT>
+int launch_router_x(const RouterParams &p, cudaStream_t st) {
+    if (p.E <= 128) return launch_router_t<XT, WT, 16>(p, st);
+    if (p.E <= 256) return launch_router_t<XT, WT, 32>(p, st);
+    return launch_router_t<XT, WT, 64>(p, st);
+}
+
+template <int KIND>
+int launch_gemm(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &a2,
+                const CUtensorMap &a3, const CUtensorMap &a4, const GemmArgs &args, int grid,
+                bool cooperative, cudaStream_t st) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(GEMM_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = GEMM_SMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = cooperative ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<KIND>, a0, a1, a2, a3, a4, args) !=
+        cudaSuccess)
+        return MOE_ERR_CUDA;
+    return launch_status();
+}
+
+int ensure_gemm_attrs(DeviceInfo *dev) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (dev->gemm_attr_set) return MOE_OK;
+    if (cudaFuncSetAttribute(grouped_gemm_kernel<GEMM_GATE_UP>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             GEMM_SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(grouped_gemm_kernel<GEMM_DOWN>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             GEMM_SMEM_BYTES) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    dev->gemm_attr_set = true;
+    return MOE_OK;
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+int moe_version(void) { return 100; }
+
+const char *moe_status_string(int status) {
+    switch (status) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_ARG: return "invalid argument (null or misaligned pointer, bad flag)";
+    case MOE_ERR_SHAPE: return "invalid or unsupported sizes";
+    case MOE_ERR_DTYPE: return "unsupported dtype combination";
+    case MOE_ERR_WORKSPACE: return "workspace missing or too small";
+    case MOE_ERR_CUDA: return "CUDA runtime error";
+    case MOE_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait ran out";
+    case MOE_ERR_BAD_INDEX: return "topk_idx held an expert id outside [0, E]";
+    case MOE_ERR_NO_DEVICE: return "no sm_100 device is current";
+    default: return "unknown status";
+    }
+}
+
+int moe_debug_set_wait_limit_ns(uint64_t ns) {
+    g_wait_limit_ns = ns ? ns : kDefaultWaitLimitNs;
+    return MOE_OK;
+}
+
+int moe_debug_never_signal(int on) {
+    g_never_signal = on ? 1 : 0;
+    return MOE_OK;
+}
+
+int moe_profile_set_events(void *const *events, int n) {
+    if (n < 0 || n > kMaxProfEvents || (n > 0 && !events)) return MOE_ERR_ARG;
+    for (int i = 0; i < n; ++i) g_prof_events[i] = events[i];
+    g_prof_n = n;
+    return MOE_OK;
+}
+
+unsigned long long moe_launch_count(void) { return g_launches.load(); }
+
+int moe_router(const void *x, int x_dtype, const void *W_g, int wg_dtype, const float *b, int N,
+               int D, int E, int n_group, int topk_group, int k, int norm_topk_prob, float alpha,
+               int32_t *topk_idx, float *topk_w, void *stream) {
+    int rc = check_router_shape(N, D, E, n_group, topk_group, k);
+    if (rc != MOE_OK) return rc;
+    if ((x_dtype != MOE_F32 && x_dtype != MOE_BF16) || (wg_dtype != MOE_F32 && wg_dtype != MOE_BF16))
+        return MOE_ERR_DTYPE;
+    if (N == 0) return MOE_OK;
+    if (!x || !W_g || !b || !topk_idx || !topk_w) return MOE_ERR_ARG;
+    if (!aligned16(x) || !aligned16(W_g) || !aligned16(b) || !aligned16(topk_idx) ||
+        !aligned16(topk_w))
+        return MOE_ERR_ARG;
+    DeviceInfo *dev = nullptr;
+    if ((rc = current_device_info(&dev)) != MOE_OK) return rc;
+    if (dev->major != 10) return MOE_ERR_NO_DEVICE;
+    RouterParams p;
+    p.x = x;
+    p.W_g = W_g;
+    p.b = b;
+    p.N = N;
+    p.D = D;
+    p.E = E;
+    p.G = n_group;
+    p.tg = topk_group;
+    p.k = k;
+    p.norm = norm_topk_prob ? 1 : 0;
+    p.alpha = alpha;
+    p.topk_idx = topk_idx;
+    p.topk_w = topk_w;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (x_dtype == MOE_F32 && wg_dtype == MOE_F32) return launch_router_x<float, float>(p, st);
+    if (x_dtype == MOE_BF16 && wg_dtype == MOE_F32) return launch_router_x<__nv_bfloat16, float>(p, st);
+    if (x_dtype == MOE_BF16 && wg_dtype == MOE_BF16)
+        return launch_router_x<__nv_bfloat16, __nv_bfloat16>(p, st);
+    return launch_router_x<float, __nv_bfloat16>(p, st);
+}
+
+size_t moe_forward_workspace(int N, int D, int E, int d_moe, int d_sh, int k, int dtype) {
+    WsLayout L;
+    if (!plan_workspace(N, D, E, d_moe, d_sh, k, dtype, L)) return 0;
+    return L.total;
+}
+
+int moe_forward(const void *x, const void *gate_up, const void *down, const void *sh_gate,
+                const void *sh_up, const void *sh_down, const int32_t *topk_idx,
+                const float *topk_w, int N, int D, int E, int d_moe, int d_sh, int k, int dtype,
+                void *y, void *workspace, size_t ws_bytes, void *stream) {
+    if (dtype != MOE_F32 && dtype != MOE_BF16) return MOE_ERR_DTYPE;
+    if (N < 0 || D <= 0 || E <= 0 || E > DISPATCH_MAXE || d_moe <= 0 || d_sh <= 0 || k <= 0 ||
+        k > 32)
+        return MOE_ERR_SHAPE;
+    if (dtype == MOE_BF16 && (D % 8 || d_moe % 8 || d_sh % 8)) return MOE_ERR_SHAPE;
+    if (dtype == MOE_F32 && (D % 4)) return MOE_ERR_SHAPE;
+    WsLayout L;
+    if (!plan_workspace(N, D, E, d_moe, d_sh, k, dtype, L)) return MOE_ERR_SHAPE;
+    if (N == 0) return MOE_OK;
+    const void *ptrs[] = {x, gate_up, down, sh_gate, sh_up, sh_down, topk_idx, topk_w, y};
+    for (const void *q : ptrs)
+        if (!q || !aligned16(q)) return MOE_ERR_ARG;
+    if (!workspace || !aligned16(workspace) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return MOE_ERR_WORKSPACE;
+    if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+    int rc;
+    DeviceInfo *dev = nullptr;
+    if ((rc = current_device_info(&dev)) != MOE_OK) return rc;
+    if (dev->major != 10) return MOE_ERR_NO_DEVICE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    Profiler prof(st);
+
+    DispatchParams dp;
+    dp.topk_idx = topk_idx;
+    dp.topk_w = topk_w;
+    dp.N = N;
+    dp.k = k;
+    dp.E = E;
+    dp.nchunks = L.nchunks;
+    dp.chunk_hist = reinterpret_cast<int32_t *>(ws + L.chunk_hist);
+    dp.counts = reinterpret_cast<int32_t *>(ws + L.counts);
+    dp.tile_off = reinterpret_cast<int32_t *>(ws + L.tile_off);
+    dp.meta = reinterpret_cast<int32_t *>(ws + L.meta);
+    dp.pos_of = reinterpret_cast<int32_t *>(ws + L.pos_of);
+    dp.perm_tok = reinterpret_cast<int32_t *>(ws + L.perm_tok);
+    dp.w_perm = reinterpret_cast<float *>(ws + L.w_perm);
+
+    dispatch_count_kernel<<<L.nchunks, DISPATCH_THREADS, 0, st>>>(dp);
+    if ((rc = launched(prof)) != MOE_OK) return rc;
+    dispatch_scan_kernel<<<1, DISPATCH_MAXE, 0, st>>>(dp);
+    if ((rc = launched(prof)) != MOE_OK) return rc;
+    dispatch_scatter_kernel<<<L.nchunks, DISPATCH_THREADS, 0, st>>>(dp);
+    if ((rc = launched(prof)) != MOE_OK) return rc;
+
+    if (dtype == MOE_F32) {
+        SimtArgs a;
+        a.x = static_cast<const float *>(x);
+        a.gate_up = static_cast<const float *>(gate_up);
+        a.down = static_cast<const float *>(down);
+        a.sh_gate = static_cast<const float *>(sh_gate);
+        a.sh_up = static_cast<const float *>(sh_up);
+        a.sh_down = static_cast<const float *>(sh_down);
+        a.perm_tok = dp.perm_tok;
+        a.tile_off = dp.tile_off;
+        a.meta = dp.meta;
+        a.pos_of = dp.pos_of;
+        a.w_perm = dp.w_perm;
+        a.h_perm = reinterpret_cast<float *>(ws + L.h_perm);
+        a.h_sh = reinterpret_cast<float *>(ws + L.h_sh);
+        a.slot = reinterpret_cast<float *>(ws + L.slot);
+        a.y = static_cast<float *>(y);
+        a.N = N;
+        a.D = D;
+        a.E = E;
+        a.d = d_moe;
+        a.d_sh = d_sh;
+        a.k = k;
+        const int rblocks = (int)(L.rows_max / SIMT_T);
+        const int nblocks = (N + SIMT_T - 1) / SIMT_T;
+        simt_expert_kernel<SIMT_GATEUP_R><<<dim3(rblocks, (d_moe + 31) / 32), 256, 0, st>>>(a);
+        if ((rc = launched(prof)) != MOE_OK) return rc;
+        simt_expert_kernel<SIMT_GATEUP_S><<<dim3(nblocks, (d_sh + 31) / 32), 256, 0, st>>>(a);
+        if ((rc = launched(prof)) != MOE_OK) return rc;
+        simt_expert_kernel<SIMT_DOWN_R><<<dim3(rblocks, (D + 31) / 32), 256, 0, st>>>(a);
+        if ((rc = launched(prof)) != MOE_OK) return rc;
+        simt_expert_kernel<SIMT_DOWN_S><<<dim3(nblocks, (D + 31) / 32), 256, 0, st>>>(a);
+        if ((rc = launched(prof)) != MOE_OK) return rc;
+        const size_t total = (size_t)N * D;
+        const int cblocks = (int)std::min<size_t>((total + 255) / 256, (size_t)dev->sms * 16);
+        simt_combine_kernel<<<cblocks, 256, 0, st>>>(a);
+        return launched(prof);
+    }
+
+    // ---- bf16 tensor-core path ----
+    uint8_t *x_perm = ws + L.x_perm;
+    {
+        const int rows = (int)L.rows_max;
+        const int grid = std::min((rows + 7) / 8, dev->sms * 16);
+        dispatch_gather_kernel<<<grid, 256, 0, st>>>(static_cast<const uint8_t *>(x), x_perm,
+                                                    dp.perm_tok, dp.meta, D * 2, rows);
+        if ((rc = launched(prof)) != MOE_OK) return rc;
+    }
+    if ((rc = ensure_gemm_attrs(dev)) != MOE_OK) return rc;
+    __nv_bfloat16 *h_perm = reinterpret_cast<__nv_bfloat16 *>(ws + L.h_perm);
+    __nv_bfloat16 *h_sh = reinterpret_cast<__nv_bfloat16 *>(ws + L.h_sh);
+    __nv_bfloat16 *slot = reinterpret_cast<__nv_bfloat16 *>(ws + L.slot);
+
+    CUtensorMap mx_perm, mgu, mx, msg, msu, mh_perm, mdn, mh_sh, msd;
+    bool ok = make_map(&mx_perm, x_perm, D, L.rows_max, D, 128) &&
+              make_map(&mgu, gate_up, D, (uint64_t)E * 2 * d_moe, D, 128) &&
+              make_map(&mx, x, D, N, D, 128) && make_map(&msg, sh_gate, D, d_sh, D, 128) &&
+              make_map(&msu, sh_up, D, d_sh, D, 128) &&
+              make_map(&mh_perm, h_perm, d_moe, L.rows_max, d_moe, 128) &&
+              make_map(&mdn, down, d_moe, (uint64_t)E * D, d_moe, GEMM_BN) &&
+              make_map(&mh_sh, h_sh, d_sh, N, d_sh, 128) &&
+              make_map(&msd, sh_down, d_sh, D, d_sh, GEMM_BN);
+    if (!ok) return MOE_ERR_CUDA;
+
+    const int mt_s = (N + GEMM_BM - 1) / GEMM_BM;
+    const int mt_r_max = (int)(L.rows_max / GEMM_BM);
+    GemmArgs g = {};
+    g.tile_off = dp.tile_off;
+    g.meta = dp.meta;
+    g.E = E;
+    g.N = N;
+    g.k = k;
+    g.mt_s = mt_s;
+    g.wait_limit_ns = g_wait_limit_ns;
+    g.never_signal = g_never_signal;
+
+    // gate_up + SwiGLU
+    g.nb_r = (d_moe + 127) / 128;
+    g.nb_s = (d_sh + 127) / 128;
+    g.kb_r = g.kb_s = (D + GEMM_BK - 1) / GEMM_BK;
+    g.b_rows_per_e = 2 * d_moe;
+    g.up_off = d_moe;
+    g.out_r = h_perm;
+    g.ld_r = d_moe;
+    g.ncols_r = d_moe;
+    g.out_s = h_sh;
+    g.ld_s = d_sh;
+    g.ncols_s = d_sh;
+    int max_tiles = mt_r_max * g.nb_r + mt_s * g.nb_s;
+    rc = launch_gemm<GEMM_GATE_UP>(mx_perm, mgu, mx, msg, msu, g, std::min(dev->sms, max_tiles),
+                                   false, st);
+    prof.mark();
+    if (rc != MOE_OK) return rc;
+
+    // down + weighted slot partials + shared expert + combine
+    g.nb_r = g.nb_s = (D + GEMM_BN - 1) / GEMM_BN;
+    g.kb_r = (d_moe + GEMM_BK - 1) / GEMM_BK;
+    g.kb_s = (d_sh + GEMM_BK - 1) / GEMM_BK;
+    g.b_rows_per_e = D;
+    g.up_off = 0;
+    g.out_r = slot;
+    g.ld_r = D;
+    g.ncols_r = D;
+    g.out_s = static_cast<__nv_bfloat16 *>(y);
+    g.ld_s = D;
+    g.ncols_s = D;
+    g.w_perm = dp.w_perm;
+    g.pos_of = dp.pos_of;
+    g.slot = slot;
+    max_tiles = mt_r_max * g.nb_r + mt_s * g.nb_s;
+    rc = launch_gemm<GEMM_DOWN>(mh_perm, mdn, mh_sh, msd, msd, g, std::min(dev->sms, max_tiles),
+                                true, st);
+    prof.mark();
+    return rc;
+}
+
+int moe_device_status(void *stream) {
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_CUDA;
+    DevStatus s;
+    if (cudaMemcpyFromSymbol(&s, g_status, sizeof(s)) != cudaSuccess) return MOE_ERR_CUDA;
+    const DevStatus zero = {0, 0, 0, 0};
+    if (cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess) return MOE_ERR_CUDA;
+    if (s.error == DEV_TIMEOUT) return MOE_ERR_DEVICE_TIMEOUT;
+    if (s.error == DEV_BAD_INDEX) return MOE_ERR_BAD_INDEX;
+    return MOE_OK;
+}
+
+}  // extern "C"

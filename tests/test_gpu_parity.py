@@ -1,0 +1,237 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle.
+
+Small cases compare every output element and span several tiles with ragged
+tails (token counts, expert loads, D, d_moe and d_sh that are not tile
+multiples).  Full-size cases use the configurations' own shapes and the same
+launch path the bench times, and compare all router ids and weights plus a
+seeded sample of output rows.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sparse_moe_layer_02_b200 as moe
+from workloads import CONFIGS, make_inputs, router_inputs
+
+from _parity import W_TOL, Y_TOL, compare_routing, rel_err
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+def _oracle_route(cfg, inp):
+    return oracle.router(inp.x, inp.W_g, inp.b, cfg.n_group, cfg.topk_group, cfg.k,
+                         cfg.norm_topk_prob, cfg.alpha)
+
+
+def _weights(inp):
+    return (inp.x, inp.gate_up, inp.down, inp.sh_gate, inp.sh_up, inp.sh_down)
+
+
+def _gpu_forward(inp_d, idx, w):
+    y = moe.moe_forward(*_weights(inp_d), idx, w)
+    assert moe.moe_device_status() == 0
+    return y
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _reset_hooks():
+    moe.moe_debug_set_wait_limit_ns(0)
+    moe.moe_debug_never_signal(False)
+    yield
+    moe.moe_debug_set_wait_limit_ns(0)
+    moe.moe_debug_never_signal(False)
+
+
+# ----------------------------------------------------------------------------- router
+@pytest.mark.parametrize("name", list(CONFIGS))
+def test_router_parity_full_size(name):
+    cfg = CONFIGS[name]
+    x, wg, b, _ = router_inputs(cfg, seed=0, device=DEV)
+    W_g = wg.to(cfg.wg_dtype)
+    idx, w = moe.moe_router(x, W_g, b, cfg.n_group, cfg.topk_group, cfg.k, cfg.norm_topk_prob,
+                            cfg.alpha)
+    assert moe.moe_device_status() == 0
+    orc = oracle.router(x.cpu(), W_g.cpu(), b.cpu(), cfg.n_group, cfg.topk_group, cfg.k,
+                        cfg.norm_topk_prob, cfg.alpha)
+    rep = compare_routing(idx, w, orc, b, cfg.alpha)
+    print(name, {k: v for k, v in rep.items() if k != "near_tie_mask"},
+          "zero-fill differs:", int(orc["zero_fill_differs"].sum()))
+    assert rep["unexplained"] == 0
+    assert rep["max_w_err_over_alpha"] <= W_TOL
+    assert int(orc["zero_fill_differs"].sum()) == 0
+
+
+@pytest.mark.parametrize("norm", [True, False])
+def test_router_group_path_and_unnormalised(norm):
+    cfg = CONFIGS["tiny_fp32"].with_(N=1000, norm_topk_prob=norm)
+    x, wg, b, _ = router_inputs(cfg, seed=5, device=DEV)
+    idx, w = moe.moe_router(x, wg, b, cfg.n_group, cfg.topk_group, cfg.k, norm, cfg.alpha)
+    orc = oracle.router(x.cpu(), wg.cpu(), b.cpu(), cfg.n_group, cfg.topk_group, cfg.k, norm,
+                        cfg.alpha)
+    rep = compare_routing(idx, w, orc, b, cfg.alpha)
+    assert rep["unexplained"] == 0 and rep["max_w_err_over_alpha"] <= W_TOL
+
+
+def test_router_bias_reorders_selection_but_not_weights():
+    # Large bias: s' order differs from s order; weights must still come from s.
+    cfg = CONFIGS["tiny_fp32"].with_(N=512, beta=0.3, n_group=1, topk_group=1)
+    x, wg, b, _ = router_inputs(cfg, seed=9, device=DEV)
+    idx, w = moe.moe_router(x, wg, b, 1, 1, cfg.k, True, cfg.alpha)
+    orc = oracle.router(x.cpu(), wg.cpu(), b.cpu(), 1, 1, cfg.k, True, cfg.alpha)
+    plain = oracle.router(x.cpu(), wg.cpu(), torch.zeros_like(b).cpu(), 1, 1, cfg.k, True, cfg.alpha)
+    assert np.any(np.sort(plain["idx"], 1) != np.sort(orc["idx"], 1))
+    rep = compare_routing(idx, w, orc, b, cfg.alpha)
+    assert rep["unexplained"] == 0 and rep["max_w_err_over_alpha"] <= W_TOL
+
+
+@pytest.mark.parametrize("E,G,tg,k", [(64, 8, 3, 6), (512, 1, 1, 8), (288, 1, 1, 8),
+                                      (256, 64, 8, 16), (160, 1, 1, 1)])
+def test_router_shapes(E, G, tg, k):
+    cfg = CONFIGS["glm5_prefill"].with_(N=333, D=264, E=E, n_group=G, topk_group=tg, k=k)
+    x, wg, b, _ = router_inputs(cfg, seed=E + k, device=DEV)
+    W_g = wg.to(torch.bfloat16)
+    idx, w = moe.moe_router(x, W_g, b, G, tg, k, True, cfg.alpha)
+    orc = oracle.router(x.cpu(), W_g.cpu(), b.cpu(), G, tg, k, True, cfg.alpha)
+    rep = compare_routing(idx, w, orc, b, cfg.alpha)
+    assert rep["unexplained"] == 0 and rep["max_w_err_over_alpha"] <= W_TOL
+
+
+# ----------------------------------------------------------------------------- forward
+SMALL = {
+    # name: (base config, overrides)
+    "bf16_tiles": ("glm5_prefill", dict(N=300, D=512, E=8, k=4, d_moe=384, d_sh=384)),
+    "bf16_ragged": ("glm5_prefill", dict(N=257, D=520, E=6, k=3, d_moe=200, d_sh=136)),
+    "bf16_group": ("skew_grouped", dict(N=200, D=256, E=32, n_group=4, topk_group=2, k=4,
+                                        d_moe=128, d_sh=256, skew=False)),
+    "bf16_single_token": ("glm5_decode", dict(N=1, D=256, E=16, k=8, d_moe=128, d_sh=128)),
+    "bf16_k1_e1": ("glm5_decode", dict(N=130, D=128, E=1, k=1, d_moe=64, d_sh=64)),
+    "fp32_tiny": ("tiny_fp32", dict()),
+    "fp32_ragged": ("tiny_fp32", dict(N=77, D=100, E=6, n_group=2, topk_group=1, k=2,
+                                      d_moe=40, d_sh=24)),
+}
+
+
+@pytest.mark.parametrize("case", list(SMALL))
+def test_forward_parity_small(case):
+    base, over = SMALL[case]
+    cfg = CONFIGS[base].with_(**over)
+    inp = make_inputs(cfg, seed=1, device="cpu")
+    orc = _oracle_route(cfg, inp)
+    y_ref = oracle.forward(*_weights(inp), orc["idx"], orc["w"])
+    inp_d = inp.to(DEV)
+    idx = torch.from_numpy(orc["idx"]).to(DEV)
+    w = torch.from_numpy(orc["w"]).float().to(DEV)
+    y = _gpu_forward(inp_d, idx, w)
+    err = rel_err(y.float().cpu().numpy(), y_ref)
+    print(case, err)
+    assert err["finite"] and err["max_rel"] <= Y_TOL[cfg.dtype]
+    # Whole layer on the GPU (router included) against the oracle end to end.
+    y2, gidx, gw = moe.moe_layer(inp_d.x, inp_d.W_g, inp_d.b, *_weights(inp_d)[1:], cfg.n_group,
+                                 cfg.topk_group, cfg.k, cfg.norm_topk_prob, cfg.alpha)
+    rep = compare_routing(gidx, gw, orc, inp.b, cfg.alpha)
+    assert rep["unexplained"] == 0
+    keep = ~rep["near_tie_mask"]
+    err2 = rel_err(y2.float().cpu().numpy()[keep], y_ref[keep])
+    assert err2["max_rel"] <= Y_TOL[cfg.dtype]
+
+
+def test_forward_sentinel_and_hot_expert():
+    cfg = CONFIGS["glm5_prefill"].with_(N=400, D=256, E=8, k=4, d_moe=128, d_sh=128)
+    inp = make_inputs(cfg, seed=2)
+    rng = np.random.default_rng(3)
+    idx = np.stack([rng.permutation(cfg.E)[:cfg.k] for _ in range(cfg.N)]).astype(np.int32)
+    idx[:, 0] = 5                 # every token hits expert 5: one expert with N rows
+    idx[::3, 2] = cfg.E           # sentinel slots are skipped
+    w = rng.uniform(0.1, 1.0, size=idx.shape)
+    y_ref = oracle.forward(*_weights(inp), idx, w)
+    y = _gpu_forward(inp.to(DEV), torch.from_numpy(idx).to(DEV), torch.from_numpy(w).float().to(DEV))
+    err = rel_err(y.float().cpu().numpy(), y_ref)
+    assert err["max_rel"] <= Y_TOL[torch.bfloat16]
+
+
+def test_forward_zero_tokens_is_noop():
+    cfg = CONFIGS["glm5_prefill"].with_(N=0, D=256, E=8, k=2, d_moe=128, d_sh=128)
+    inp = make_inputs(cfg, seed=0, device=DEV)
+    idx = torch.empty((0, 2), dtype=torch.int32, device=DEV)
+    w = torch.empty((0, 2), dtype=torch.float32, device=DEV)
+    y = moe.moe_forward(*_weights(inp), idx, w)
+    assert y.shape == (0, 256)
+    i2, w2 = moe.moe_router(inp.x, inp.W_g, inp.b, 1, 1, 2, True, 2.5)
+    assert i2.shape == (0, 2)
+    assert moe.moe_device_status() == 0
+
+
+def test_forward_is_deterministic():
+    cfg = CONFIGS["glm5_prefill"].with_(N=1000, D=512, E=16, k=8, d_moe=256, d_sh=256)
+    inp = make_inputs(cfg, seed=4, device=DEV)
+    y1, _, _ = moe.moe_layer(inp.x, inp.W_g, inp.b, *_weights(inp)[1:], 1, 1, 8, True, 2.5)
+    y2, _, _ = moe.moe_layer(inp.x, inp.W_g, inp.b, *_weights(inp)[1:], 1, 1, 8, True, 2.5)
+    assert torch.equal(y1, y2)
+
+
+def test_bad_expert_id_is_skipped_and_reported():
+    cfg = CONFIGS["glm5_prefill"].with_(N=64, D=256, E=8, k=2, d_moe=128, d_sh=128)
+    inp = make_inputs(cfg, seed=6)
+    rng = np.random.default_rng(7)
+    idx = np.stack([rng.permutation(cfg.E)[:2] for _ in range(cfg.N)]).astype(np.int32)
+    w = rng.uniform(0.1, 1.0, size=idx.shape)
+    bad = idx.copy()
+    bad[5, 1] = cfg.E + 3
+    w0 = w.copy()
+    w0[5, 1] = 0.0
+    y_ref = oracle.forward(*_weights(inp), idx, w0)
+    y = moe.moe_forward(*_weights(inp.to(DEV)), torch.from_numpy(bad).to(DEV),
+                        torch.from_numpy(w).float().to(DEV))
+    assert moe.moe_device_status() == -7
+    assert rel_err(y.float().cpu().numpy(), y_ref)["max_rel"] <= Y_TOL[torch.bfloat16]
+    assert moe.moe_device_status() == 0  # cleared
+
+
+def test_bounded_wait_times_out_and_context_survives():
+    cfg = CONFIGS["glm5_prefill"].with_(N=256, D=256, E=8, k=2, d_moe=128, d_sh=128)
+    inp = make_inputs(cfg, seed=8, device=DEV)
+    idx, w = moe.moe_router(inp.x, inp.W_g, inp.b, 1, 1, 2, True, 2.5)
+    moe.moe_debug_set_wait_limit_ns(20_000_000)
+    moe.moe_debug_never_signal(True)
+    try:
+        moe.moe_forward(*_weights(inp), idx, w)
+        assert moe.moe_device_status() == -6
+    finally:
+        moe.moe_debug_never_signal(False)
+        moe.moe_debug_set_wait_limit_ns(0)
+    y = _gpu_forward(inp, idx, w)
+    orc_idx, orc_w = idx.cpu().numpy(), w.cpu().double().numpy()
+    y_ref = oracle.forward(*_weights(inp.to("cpu")), orc_idx, orc_w)
+    assert rel_err(y.float().cpu().numpy(), y_ref)["max_rel"] <= Y_TOL[torch.bfloat16]
+
+
+# ----------------------------------------------------------------------------- full size
+FULL = ["air_decode", "glm5_decode", "glm45_prefill", "glm5_prefill", "skew_grouped"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_layer_parity_full_size_sampled(name):
+    cfg = CONFIGS[name]
+    inp = make_inputs(cfg, seed=0, device=DEV)
+    y, idx, w = moe.moe_layer(inp.x, inp.W_g, inp.b, *_weights(inp)[1:], cfg.n_group,
+                              cfg.topk_group, cfg.k, cfg.norm_topk_prob, cfg.alpha)
+    assert moe.moe_device_status() == 0
+    host = inp.to("cpu")
+    orc = _oracle_route(cfg, host)
+    rep = compare_routing(idx, w, orc, host.b, cfg.alpha)
+    assert rep["unexplained"] == 0 and rep["max_w_err_over_alpha"] <= W_TOL
+    rng = np.random.default_rng(0)
+    cand = np.nonzero(~rep["near_tie_mask"])[0]
+    sample = np.sort(rng.choice(cand, size=min(len(cand), 24), replace=False)).astype(np.int32)
+    y_ref = oracle.forward(*_weights(host), orc["idx"], orc["w"], tokens=sample)
+    err = rel_err(y[torch.from_numpy(sample).long().to(DEV)].float().cpu().numpy(), y_ref)
+    loads = np.bincount(idx.cpu().numpy().ravel(), minlength=cfg.E)
+    print(name, err, "hit experts:", int((loads > 0).sum()), "max/mean load:",
+          float(loads.max() / loads.mean()), "near ties:", rep["near_tie_tokens"])
+    assert err["finite"] and err["max_rel"] <= Y_TOL[cfg.dtype]
+    if cfg.skew:
+        assert loads.max() / loads.mean() > 5.0
