@@ -94,6 +94,13 @@ class ClockSampler:
                 stdout=self.out, stderr=subprocess.DEVNULL)
         except (OSError, ValueError):
             self.proc = None
+            return
+        # Do not start timing before the sampler produces its first line.
+        t0 = time.time()
+        while time.time() - t0 < 10.0 and self.proc.poll() is None:
+            if os.path.getsize(self.path) > 0:
+                break
+            time.sleep(0.05)
 
     def stop(self):
         if self.proc is None:
@@ -308,7 +315,6 @@ def main():
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
-    clocks = sampler.stop()
     status = moe.moe_device_status(stream)
     if status != 0:
         raise SystemExit("device status after timing: %s" % moe.moe_status_string(status))
@@ -367,6 +373,7 @@ def main():
         dist.all_reduce(et, op=dist.ReduceOp.MAX)
     e2e_value = N * world * K / (float(et.item()) / 1e3)
     es = inp.x.element_size()
+    clocks = sampler.stop()
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
