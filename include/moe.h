@@ -113,6 +113,36 @@ int moe_forward(const void *x, const void *gate_up, const void *down, const void
                 const float *topk_w, int N, int D, int E, int d_moe, int d_sh, int k,
                 int dtype, void *y, void *workspace, size_t ws_bytes, void *stream);
 
+/* Bytes of device scratch built into the library for moe_forward_noalloc. */
+#define MOE_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+
+/*
+ * moe_forward_noalloc — moe_forward for callers that cannot allocate device
+ * memory.  The pages have no counterpart; this is a deployment aid.
+ *
+ * Some callers have no way to call cudaMalloc on the hot path.  A plugin inside
+ * a serving runtime that owns every device allocation is one.  A
+ * latency-critical loop that must not call cudaMalloc, because cudaMalloc can
+ * synchronise the device, is another.  This entry point takes the same
+ * arguments as moe_forward minus the workspace.  It uses a scratch array of
+ * MOE_NOALLOC_SCRATCH_BYTES (64 MiB) that the library holds in device memory on
+ * every GPU that loads it, until the process exits.  It calls no allocator.
+ *   - Sizes whose moe_forward_workspace() exceeds MOE_NOALLOC_SCRATCH_BYTES are
+ *     refused with MOE_ERR_WORKSPACE before any launch (small layers, e.g.
+ *     N*k + 127*E up to a few thousand rows at D of a few hundred, fit).
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current.  Make it before any
+ *     stream capture.
+ *   - All calls on a device share the array, which keeps the last call's
+ *     contents.  Each call rewrites everything it reads before reading it.
+ *     Calls whose kernels overlap on the GPU race; serialise them (one stream).
+ * Results equal moe_forward's for the same inputs.
+ */
+int moe_forward_noalloc(const void *x, const void *gate_up, const void *down,
+                        const void *sh_gate, const void *sh_up, const void *sh_down,
+                        const int32_t *topk_idx, const float *topk_w, int N, int D, int E,
+                        int d_moe, int d_sh, int k, int dtype, void *y, void *stream);
+
 /*
  * moe_device_status — synchronises `stream`, then returns and clears the device
  * status word: MOE_OK, MOE_ERR_DEVICE_TIMEOUT (a bounded wait ran out; the

@@ -19,7 +19,8 @@ import torch
 
 __all__ = ["MoEError", "moe_router", "moe_forward", "moe_forward_workspace", "moe_layer",
            "moe_device_status", "moe_status_string", "moe_debug_set_wait_limit_ns",
-           "moe_debug_never_signal", "moe_profile_set_events", "moe_launch_count", "library_path", "load_library", "MOE_F32", "MOE_BF16",
+           "moe_debug_never_signal", "moe_profile_set_events", "moe_launch_count",
+           "moe_forward_noalloc", "library_path", "load_library", "MOE_F32", "MOE_BF16",
            "EXPORTED_SYMBOLS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -32,7 +33,8 @@ MOE_OK = 0
 
 EXPORTED_SYMBOLS = ("moe_router", "moe_forward_workspace", "moe_forward", "moe_device_status",
                     "moe_status_string", "moe_version", "moe_debug_set_wait_limit_ns",
-                    "moe_debug_never_signal", "moe_profile_set_events", "moe_launch_count")
+                    "moe_debug_never_signal", "moe_profile_set_events", "moe_launch_count",
+                    "moe_forward_noalloc")
 
 
 class MoEError(RuntimeError):
@@ -77,6 +79,8 @@ def load_library():
         lib.moe_profile_set_events.restype = I
         lib.moe_launch_count.argtypes = []
         lib.moe_launch_count.restype = ctypes.c_ulonglong
+        lib.moe_forward_noalloc.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, P, P]
+        lib.moe_forward_noalloc.restype = I
         _lib = lib
         return lib
 
@@ -172,6 +176,24 @@ def moe_forward(x, gate_up, down, sh_gate, sh_up, sh_down, topk_idx, topk_w, y=N
                          _dt(x), _dev(y, "y"), _dev(workspace, "workspace"),
                          workspace.numel() * workspace.element_size(), _stream(stream))
     _check(rc, "moe_forward")
+    return y
+
+
+def moe_forward_noalloc(x, gate_up, down, sh_gate, sh_up, sh_down, topk_idx, topk_w, y,
+                        stream=None):
+    """moe_forward without a workspace, for callers that cannot allocate device memory:
+    the library's built-in 64 MiB device scratch is used instead (small layers only;
+    larger ones raise with the workspace error).  y must be preallocated."""
+    lib = load_library()
+    N, D = x.shape
+    E, two_d, _ = gate_up.shape
+    k = topk_idx.shape[1]
+    rc = lib.moe_forward_noalloc(_dev(x, "x"), _dev(gate_up, "gate_up"), _dev(down, "down"),
+                                 _dev(sh_gate, "sh_gate"), _dev(sh_up, "sh_up"),
+                                 _dev(sh_down, "sh_down"), _dev(topk_idx, "topk_idx"),
+                                 _dev(topk_w, "topk_w"), N, D, E, two_d // 2, sh_gate.shape[0], k,
+                                 _dt(x), _dev(y, "y"), _stream(stream))
+    _check(rc, "moe_forward_noalloc")
     return y
 
 

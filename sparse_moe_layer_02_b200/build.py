@@ -2,9 +2,9 @@
 
     python -m sparse_moe_layer_02_b200.build [--verbose-ptxas]
 
-The library is one translation unit (csrc/moe.cu includes the kernel headers),
-linked against the static CUDA runtime so it carries no dependency on a
-particular libcudart next to torch's.
+The library is csrc/moe.cu (which includes the kernel headers) plus
+csrc/moe_noalloc.cu, linked against the static CUDA runtime so it carries no
+dependency on a particular libcudart next to torch's.
 """
 
 from __future__ import annotations
@@ -44,7 +44,8 @@ def build(force: bool = False, verbose_ptxas: bool = False) -> str:
         return LIB
     nvcc = os.environ.get("NVCC", "nvcc")
     tmp = LIB + ".tmp.%d" % os.getpid()
-    cmd = [nvcc, *NVCC_FLAGS, "-I", INCLUDE, "-o", tmp, os.path.join(CSRC, "moe.cu")]
+    cmd = [nvcc, *NVCC_FLAGS, "-I", INCLUDE, "-o", tmp, os.path.join(CSRC, "moe.cu"),
+           os.path.join(CSRC, "moe_noalloc.cu")]
     if verbose_ptxas:
         cmd[1:1] = ["-Xptxas", "-v"]
     subprocess.run(cmd, check=True)
