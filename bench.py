@@ -57,7 +57,19 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target duration of the oracle's CPU-baseline sample")
+    ap.add_argument("--set", action="append", default=[], metavar="FIELD=VALUE",
+                    help="override a size of the workload (e.g. E=32) for small profiling cases")
     return ap.parse_args()
+
+
+def workload(args):
+    cfg = CONFIGS[args.workload]
+    over = {}
+    for item in args.set:
+        key, val = item.split("=", 1)
+        cur = getattr(cfg, key)
+        over[key] = type(cur)(float(val)) if isinstance(cur, (int, float)) else val
+    return cfg.with_(**over) if over else cfg, over
 
 
 def load_peaks():
@@ -194,7 +206,7 @@ def run_reference(args):
         return
     import oracle
 
-    cfg = CONFIGS[args.workload]
+    cfg, over = workload(args)
     gen_dev = "cuda:0" if torch.cuda.is_available() else "cpu"
     inp = make_inputs(cfg, seed=0, device=gen_dev).to("cpu")
     cores = oracle.num_threads()
@@ -226,7 +238,7 @@ def run_reference(args):
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": cfg.name, "description": cfg.description, "N": cfg.N,
                        "D": cfg.D, "E": cfg.E, "k": cfg.k, "d_moe": cfg.d_moe,
-                       "sample_tokens_per_step": sample},
+                       "sample_tokens_per_step": sample, "overrides": over or None},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                              "sample": desc},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -253,7 +265,7 @@ def main():
 
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
 
-    cfg = CONFIGS[args.workload]
+    cfg, over = workload(args)
     inp = make_inputs(cfg, seed=0, device=dev)
     if rank > 0:  # each replica gets its own batch of tokens
         from workloads import make_tokens
@@ -401,6 +413,7 @@ def main():
                    "d_moe": cfg.d_moe, "d_sh": cfg.d_sh, "alpha": cfg.alpha,
                    "router_dtype": str(cfg.wg_dtype).replace("torch.", ""),
                    "hit_experts": hit, "max_over_mean_load": max_over_mean,
+                   "overrides": over or None,
                    "parallelism": "replicas" if world > 1 else "single",
                    "l2": "inputs larger than L2 (hit-expert weights %.2f GB per step)"
                          % (kernel_work(cfg, "gate_up_swiglu", hit)[1] / 1e9
