@@ -30,8 +30,8 @@ struct DispatchParams {
     int32_t *tile_off;   // [E+1] prefix of 128-row tiles per expert
     int32_t *meta;       // [0] done counter, [1] padded rows, [2] routed m-tiles
     int32_t *pos_of;     // [N*k] permuted row of each (token, slot), -1 if none
-    int32_t *perm_tok;   // [rows_max] token of each permuted row, -1 for padding
-    float *w_perm;       // [rows_max] routing weight of each permuted row, 0 for padding
+    int32_t *perm_tok;   // [rows_max] token of each permuted row (padding rows: unset)
+    float *w_perm;       // [rows_max] routing weight of each permuted row (padding rows: unset)
 };
 
 __global__ void __launch_bounds__(DISPATCH_THREADS) dispatch_count_kernel(const DispatchParams p) {
@@ -93,10 +93,6 @@ __global__ void __launch_bounds__(DISPATCH_MAXE) dispatch_scan_kernel(const Disp
         p.tile_off[e] = excl;
         const int row0 = excl * TILE_M;
         for (int c = 0; c < p.nchunks; ++c) p.chunk_hist[(size_t)c * p.E + e] += row0;
-        for (int r = row0 + total; r < row0 + tiles * TILE_M; ++r) {
-            p.perm_tok[r] = -1;
-            p.w_perm[r] = 0.f;
-        }
     }
     if (e == p.E - 1) {
         p.tile_off[p.E] = incl;
@@ -157,19 +153,37 @@ __global__ void __launch_bounds__(DISPATCH_THREADS) dispatch_scatter_kernel(cons
     }
 }
 
+// Padding rows (beyond an expert's count inside its last 128-row tile) carry no
+// token; perm_tok / w_perm are left unset there and every reader checks this.
+__device__ __forceinline__ int expert_of_tile(const int *tile_off, int E, int mt) {
+    int lo = 0, hi = E - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (tile_off[mid] <= mt) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
 // Copy x[perm_tok[r]] to x_perm[r] for every real permuted row; one warp per row,
 // 16-byte vectors.  row_bytes is a multiple of 16.
 __global__ void __launch_bounds__(256) dispatch_gather_kernel(const uint8_t *__restrict__ x,
                                                               uint8_t *__restrict__ x_perm,
-                                                              const int32_t *perm_tok,
-                                                              const int32_t *meta,
+                                                              const DispatchParams p,
                                                               int row_bytes, int rows_max) {
-    const int rows = min(meta[1], rows_max);
+    __shared__ int s_off[DISPATCH_MAXE + 1];
+    __shared__ int s_cnt[DISPATCH_MAXE];
+    for (int e = threadIdx.x; e <= p.E; e += blockDim.x) {
+        s_off[e] = p.tile_off[e];
+        if (e < p.E) s_cnt[e] = p.counts[e];
+    }
+    __syncthreads();
+    const int rows = min(s_off[p.E] * TILE_M, rows_max);
     const int lane = threadIdx.x & 31;
     for (int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < rows;
          r += (gridDim.x * blockDim.x) >> 5) {
-        const int tok = perm_tok[r];
-        if (tok < 0) continue;
+        const int e = expert_of_tile(s_off, p.E, r / TILE_M);
+        if (r - s_off[e] * TILE_M >= s_cnt[e]) continue; // padding row
+        const int tok = p.perm_tok[r];
         const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)tok * row_bytes);
         uint4 *dst = reinterpret_cast<uint4 *>(x_perm + (size_t)r * row_bytes);
         const int nvec = row_bytes >> 4;

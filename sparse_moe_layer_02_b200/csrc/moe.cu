@@ -165,30 +165,39 @@ int launched(Profiler &prof) {
     return rc;
 }
 
-template <typename XT, typename WT, int TE>
+template <typename XT, typename WT, int EV>
 int launch_router_t(const RouterParams &p, cudaStream_t st) {
-    const int CL = (p.E + TE - 1) / TE;
+    constexpr int smem = router_smem_bytes(EV);
+    static bool attr_set = false; // per process; the attribute is per function
+    if (!attr_set) {
+        if (cudaFuncSetAttribute(router_kernel<XT, WT, EV>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        attr_set = true;
+    }
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(CL, (p.N + ROUTER_TM - 1) / ROUTER_TM, 1);
+    cfg.gridDim = dim3(ROUTER_CL, (p.N + ROUTER_TM - 1) / ROUTER_TM, 1);
     cfg.blockDim = dim3(ROUTER_THREADS, 1, 1);
-    cfg.dynamicSmemBytes = 0;
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = CL;
+    attr[0].val.clusterDim.x = ROUTER_CL;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, router_kernel<XT, WT, TE>, p) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, router_kernel<XT, WT, EV>, p) != cudaSuccess) return MOE_ERR_CUDA;
     return launch_status();
 }
 
 template <typename XT, typename WT>
 int launch_router_x(const RouterParams &p, cudaStream_t st) {
-    if (p.E <= 128) return launch_router_t<XT, WT, 16>(p, st);
-    if (p.E <= 256) return launch_router_t<XT, WT, 32>(p, st);
-    return launch_router_t<XT, WT, 64>(p, st);
+    if (p.E <= 32) return launch_router_t<XT, WT, 1>(p, st);
+    if (p.E <= 64) return launch_router_t<XT, WT, 2>(p, st);
+    if (p.E <= 128) return launch_router_t<XT, WT, 4>(p, st);
+    if (p.E <= 256) return launch_router_t<XT, WT, 8>(p, st);
+    return launch_router_t<XT, WT, 16>(p, st);
 }
 
 template <int KIND>
@@ -369,6 +378,7 @@ int moe_forward(const void *x, const void *gate_up, const void *down, const void
         a.sh_up = static_cast<const float *>(sh_up);
         a.sh_down = static_cast<const float *>(sh_down);
         a.perm_tok = dp.perm_tok;
+        a.counts = dp.counts;
         a.tile_off = dp.tile_off;
         a.meta = dp.meta;
         a.pos_of = dp.pos_of;
@@ -404,8 +414,8 @@ int moe_forward(const void *x, const void *gate_up, const void *down, const void
     {
         const int rows = (int)L.rows_max;
         const int grid = std::min((rows + 7) / 8, dev->sms * 16);
-        dispatch_gather_kernel<<<grid, 256, 0, st>>>(static_cast<const uint8_t *>(x), x_perm,
-                                                    dp.perm_tok, dp.meta, D * 2, rows);
+        dispatch_gather_kernel<<<grid, 256, 0, st>>>(static_cast<const uint8_t *>(x), x_perm, dp,
+                                                    D * 2, rows);
         if ((rc = launched(prof)) != MOE_OK) return rc;
     }
     if ((rc = ensure_gemm_attrs(dev)) != MOE_OK) return rc;

@@ -1,13 +1,15 @@
 // Router: fp32 logits, sigmoid, correction bias, group top-2 score, group keep,
 // top-k and weights ("GLM-4.5 Group Router", How it works).
 //
-// One thread-block cluster handles 32 tokens.  CTA r of the cluster computes the
-// logits of experts [r*TE, r*TE + TE) for those tokens on CUDA cores (fp32 FMA;
-// bf16 and fp32 inputs are widened exactly, so every product is exact in fp32)
-// and keeps them in its shared memory.  After a cluster barrier each warp takes
-// whole tokens and reads the token's E logits from all CTAs of the cluster
-// through distributed shared memory; selection then runs in the warp's
-// registers with shuffles: lane l holds experts l, l+32, l+64, ...
+// One thread-block cluster of ROUTER_CL CTAs handles 32 tokens.  CTA r of the
+// cluster computes partial logits of all E experts for those tokens over the
+// r-th slice of the hidden dimension D, on CUDA cores in fp32 (bf16 and fp32
+// inputs are widened exactly, so every product is exact in fp32), and keeps the
+// 32 x E partial tile in its shared memory.  After a cluster barrier, warp w of
+// CTA r takes token j = r + ROUTER_CL * w: lane l sums expert l, l+32, ...
+// over the ROUTER_CL partial tiles in rank order (distributed shared memory, a
+// fixed order, so the result is deterministic) and selection then runs in the
+// warp's registers with shuffles.
 #pragma once
 
 #include <cooperative_groups.h>
@@ -18,11 +20,12 @@ namespace moe {
 
 namespace cg = cooperative_groups;
 
-constexpr int ROUTER_TM = 32;       // tokens per cluster
-constexpr int ROUTER_KC = 32;       // K chunk staged in shared memory
-constexpr int ROUTER_THREADS = 128; // 4 warps
-constexpr int ROUTER_MAXV = 16;     // experts per lane: E <= 512
-constexpr int ROUTER_MAXG = 64;     // groups
+constexpr int ROUTER_TM = 32;        // tokens per cluster
+constexpr int ROUTER_CL = 8;         // CTAs per cluster = K slices
+constexpr int ROUTER_KC = 32;        // K chunk staged in shared memory
+constexpr int ROUTER_THREADS = 256;  // 8 warps
+constexpr int ROUTER_MAXV = 16;      // experts per lane: E <= 512
+constexpr int ROUTER_MAXG = 64;      // groups
 
 struct RouterParams {
     const void *x;
@@ -33,6 +36,13 @@ struct RouterParams {
     int32_t *topk_idx;
     float *topk_w;
 };
+
+// Dynamic shared memory of router_kernel<EV>: x chunk, W chunk, partial logits,
+// per-warp s' rows for the group stage.
+__host__ __device__ constexpr int router_smem_bytes(int EV) {
+    return (ROUTER_TM * (ROUTER_KC + 1) + 32 * EV * (ROUTER_KC + 1) + ROUTER_TM * 32 * EV +
+            (ROUTER_THREADS / 32) * ROUTER_MAXV * 32) * 4;
+}
 
 // (value, index) comparison: larger value wins, ties go to the lower index.
 __device__ __forceinline__ bool better(float v, int i, float bv, int bi) {
@@ -51,79 +61,113 @@ __device__ __forceinline__ void warp_argmax(float &v, int &i) {
     }
 }
 
-template <typename XT, typename WT, int TE>
+// EV = experts per lane (E <= 32 * EV); each thread accumulates 4 tokens x EV experts.
+template <typename XT, typename WT, int EV>
 __global__ void __launch_bounds__(ROUTER_THREADS)
     router_kernel(const RouterParams p) {
-    constexpr int EPT = TE / 8; // experts per thread in the logits tile
-    __shared__ float xs[ROUTER_TM][ROUTER_KC + 1];
-    __shared__ float ws[TE][ROUTER_KC + 1];
-    __shared__ float logit[ROUTER_TM][TE];
-    __shared__ float spbuf[4][ROUTER_MAXV * 32];
+    extern __shared__ float rsm[];
+    float(*xs)[ROUTER_KC + 1] = reinterpret_cast<float(*)[ROUTER_KC + 1]>(rsm);
+    float(*ws)[ROUTER_KC + 1] =
+        reinterpret_cast<float(*)[ROUTER_KC + 1]>(rsm + ROUTER_TM * (ROUTER_KC + 1));
+    float *part = rsm + ROUTER_TM * (ROUTER_KC + 1) + 32 * EV * (ROUTER_KC + 1); // [TM][32*EV]
+    float *spbuf = part + ROUTER_TM * 32 * EV; // [8 warps][MAXV*32]
+    constexpr int EP = 32 * EV;                // padded expert count
 
     cg::cluster_group cluster = cg::this_cluster();
-    const int CL = gridDim.x;
     const int rank = blockIdx.x;
     const int t0 = blockIdx.y * ROUTER_TM;
-    const int e0 = rank * TE;
-    const int tid = threadIdx.x;
-    const int ty = tid >> 3, tx = tid & 7;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int E = p.E;
+
+    // K slice of this CTA (a multiple of the chunk size).
+    const int kper = ((p.D + ROUTER_CL * ROUTER_KC - 1) / (ROUTER_CL * ROUTER_KC)) * ROUTER_KC;
+    const int kbeg = rank * kper, kend = min(p.D, kbeg + kper);
 
     const XT *x = static_cast<const XT *>(p.x);
     const WT *W = static_cast<const WT *>(p.W_g);
 
-    // ---- logits tile [32 tokens x TE experts], fp32 accumulation -------------
-    float acc0[EPT], acc1[EPT];
+    // ---- partial logits [32 tokens x E] over [kbeg, kend) ----------------------
+    // thread: tokens warp + 8*i (i < 4), experts lane + 32*j (j < EV)
+    float acc[4][EV];
 #pragma unroll
-    for (int j = 0; j < EPT; ++j) acc0[j] = acc1[j] = 0.f;
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < EV; ++j) acc[i][j] = 0.f;
 
-    for (int k0 = 0; k0 < p.D; k0 += ROUTER_KC) {
-        for (int i = tid; i < ROUTER_TM * ROUTER_KC; i += ROUTER_THREADS) {
+    // Register-staged double buffering: the next chunk's loads are in flight
+    // while the current chunk is multiplied out of shared memory.
+    constexpr int XPT = ROUTER_TM * ROUTER_KC / ROUTER_THREADS; // 4
+    constexpr int WPT = EP * ROUTER_KC / ROUTER_THREADS;        // 4 * EV
+    float xr[XPT], wr[WPT];
+    auto load_chunk = [&](int k0) {
+#pragma unroll
+        for (int q = 0; q < XPT; ++q) {
+            const int i = tid + ROUTER_THREADS * q;
             const int r = i / ROUTER_KC, c = i % ROUTER_KC;
             const int t = t0 + r, kk = k0 + c;
-            xs[r][c] = (t < p.N && kk < p.D) ? to_f32(x[(size_t)t * p.D + kk]) : 0.f;
+            xr[q] = (t < p.N && kk < kend) ? to_f32(x[(size_t)t * p.D + kk]) : 0.f;
         }
-        for (int i = tid; i < TE * ROUTER_KC; i += ROUTER_THREADS) {
+#pragma unroll
+        for (int q = 0; q < WPT; ++q) {
+            const int i = tid + ROUTER_THREADS * q;
             const int r = i / ROUTER_KC, c = i % ROUTER_KC;
-            const int e = e0 + r, kk = k0 + c;
-            ws[r][c] = (e < p.E && kk < p.D) ? to_f32(W[(size_t)e * p.D + kk]) : 0.f;
+            const int kk = k0 + c;
+            wr[q] = (r < E && kk < kend) ? to_f32(W[(size_t)r * p.D + kk]) : 0.f;
+        }
+    };
+    if (kbeg < kend) load_chunk(kbeg);
+    for (int k0 = kbeg; k0 < kend; k0 += ROUTER_KC) {
+#pragma unroll
+        for (int q = 0; q < XPT; ++q) {
+            const int i = tid + ROUTER_THREADS * q;
+            xs[i / ROUTER_KC][i % ROUTER_KC] = xr[q];
+        }
+#pragma unroll
+        for (int q = 0; q < WPT; ++q) {
+            const int i = tid + ROUTER_THREADS * q;
+            ws[i / ROUTER_KC][i % ROUTER_KC] = wr[q];
         }
         __syncthreads();
-#pragma unroll 8
+        if (k0 + ROUTER_KC < kend) load_chunk(k0 + ROUTER_KC);
+#pragma unroll 4
         for (int kk = 0; kk < ROUTER_KC; ++kk) {
-            const float a0 = xs[ty][kk], a1 = xs[ty + 16][kk];
+            float a[4], w[EV];
 #pragma unroll
-            for (int j = 0; j < EPT; ++j) {
-                const float w = ws[tx + 8 * j][kk];
-                acc0[j] = fmaf(a0, w, acc0[j]);
-                acc1[j] = fmaf(a1, w, acc1[j]);
-            }
+            for (int i = 0; i < 4; ++i) a[i] = xs[warp + 8 * i][kk];
+#pragma unroll
+            for (int j = 0; j < EV; ++j) w[j] = ws[lane + 32 * j][kk];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < EV; ++j) acc[i][j] = fmaf(a[i], w[j], acc[i][j]);
         }
         __syncthreads();
     }
 #pragma unroll
-    for (int j = 0; j < EPT; ++j) {
-        logit[ty][tx + 8 * j] = acc0[j];
-        logit[ty + 16][tx + 8 * j] = acc1[j];
-    }
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < EV; ++j) part[(warp + 8 * i) * EP + lane + 32 * j] = acc[i][j];
     cluster.sync();
 
-    // ---- selection: one warp per token --------------------------------------
-    const int warp = tid >> 5, lane = tid & 31;
-    const int E = p.E, G = p.G, m = E / G;
-    const int V = (E + 31) >> 5;
-    float *sp_w = spbuf[warp];
-    for (int j = rank + CL * warp; j < ROUTER_TM; j += CL * 4) {
-        const int t = t0 + j;
-        if (t >= p.N) break;
-        float s[ROUTER_MAXV], sp[ROUTER_MAXV];
+    // ---- reduce over the cluster's K slices, then select: one warp per token ----
+    const int G = p.G, m = E / G;
+    const int j = rank + ROUTER_CL * warp; // token of this warp (32 = CL * 4 tokens per cluster)
+    const int t = t0 + j;
+    if (warp < ROUTER_TM / ROUTER_CL && t < p.N) {
+        float *sp_w = spbuf + warp * ROUTER_MAXV * 32;
+        float s[EV], sp[EV];
 #pragma unroll
-        for (int v = 0; v < ROUTER_MAXV; ++v) {
+        for (int v = 0; v < EV; ++v) {
             const int e = lane + 32 * v;
             s[v] = 0.f;
             sp[v] = -INFINITY;
-            if (v < V && e < E) {
-                const float *remote = cluster.map_shared_rank(&logit[0][0], e / TE);
-                const float r = remote[j * TE + (e % TE)];
+            if (e < E) {
+                float r = 0.f;
+#pragma unroll
+                for (int c = 0; c < ROUTER_CL; ++c) {
+                    const float *remote = cluster.map_shared_rank(part, c);
+                    r += remote[j * EP + e];
+                }
                 s[v] = 1.0f / (1.0f + expf(-r));
                 sp[v] = s[v] + p.b[e];
             }
@@ -132,10 +176,10 @@ __global__ void __launch_bounds__(ROUTER_THREADS)
         uint32_t cand = 0;
         if (G > 1) {
 #pragma unroll
-            for (int v = 0; v < ROUTER_MAXV; ++v)
-                if (v < V && lane + 32 * v < E) sp_w[lane + 32 * v] = sp[v];
+            for (int v = 0; v < EV; ++v)
+                if (lane + 32 * v < E) sp_w[lane + 32 * v] = sp[v];
             __syncwarp();
-            // Group score = sum of the two largest s' of the group (lane g, g+32).
+            // Group score = sum of the two largest s' of the group (lanes own g, g+32).
             float gs[2] = {-INFINITY, -INFINITY};
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
@@ -171,14 +215,14 @@ __global__ void __launch_bounds__(ROUTER_THREADS)
                 kept |= 1ull << bi;
             }
 #pragma unroll
-            for (int v = 0; v < ROUTER_MAXV; ++v) {
+            for (int v = 0; v < EV; ++v) {
                 const int e = lane + 32 * v;
-                if (v < V && e < E && ((kept >> (e / m)) & 1ull)) cand |= 1u << v;
+                if (e < E && ((kept >> (e / m)) & 1ull)) cand |= 1u << v;
             }
         } else {
 #pragma unroll
-            for (int v = 0; v < ROUTER_MAXV; ++v)
-                if (v < V && lane + 32 * v < E) cand |= 1u << v;
+            for (int v = 0; v < EV; ++v)
+                if (lane + 32 * v < E) cand |= 1u << v;
         }
         // Top-k by s' among candidates; lane r keeps the r-th pick.
         int my_e = -1;
@@ -187,7 +231,7 @@ __global__ void __launch_bounds__(ROUTER_THREADS)
             float bv = -INFINITY;
             int bi = 0x7fffffff;
 #pragma unroll
-            for (int v = 0; v < ROUTER_MAXV; ++v) {
+            for (int v = 0; v < EV; ++v) {
                 if ((cand >> v) & 1u) {
                     const int e = lane + 32 * v;
                     if (better(sp[v], e, bv, bi)) {
@@ -200,7 +244,7 @@ __global__ void __launch_bounds__(ROUTER_THREADS)
             const int owner = bi & 31, vw = bi >> 5;
             float sv = 0.f;
 #pragma unroll
-            for (int v = 0; v < ROUTER_MAXV; ++v)
+            for (int v = 0; v < EV; ++v)
                 if (v == vw) sv = s[v];
             sv = __shfl_sync(0xffffffffu, sv, owner);
             if (lane == owner) cand &= ~(1u << vw);
@@ -219,7 +263,7 @@ __global__ void __launch_bounds__(ROUTER_THREADS)
             p.topk_w[(size_t)t * p.k + lane] = w;
         }
     }
-    cluster.sync(); // keep this CTA's logits alive until every reader is done
+    cluster.sync(); // keep this CTA's partials alive until every reader is done
 }
 
 }  // namespace moe

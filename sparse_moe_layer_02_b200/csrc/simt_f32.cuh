@@ -18,7 +18,7 @@ enum SimtMode { SIMT_GATEUP_R = 0, SIMT_GATEUP_S = 1, SIMT_DOWN_R = 2, SIMT_DOWN
 
 struct SimtArgs {
     const float *x, *gate_up, *down, *sh_gate, *sh_up, *sh_down;
-    const int32_t *perm_tok, *tile_off, *meta, *pos_of;
+    const int32_t *perm_tok, *counts, *tile_off, *meta, *pos_of;
     const float *w_perm;
     float *h_perm, *h_sh, *slot, *y;
     int N, D, E, d, d_sh, k;
@@ -48,6 +48,8 @@ __global__ void __launch_bounds__(256) simt_expert_kernel(const SimtArgs a) {
     const int ncols = GATEUP ? (ROUTED ? a.d : a.d_sh) : a.D;
     const int K = GATEUP ? a.D : (ROUTED ? a.d : a.d_sh);
     const int e = ROUTED ? expert_of_row(a.tile_off, a.E, r0) : 0;
+    // Rows of expert e at or beyond seg_end are padding (no token).
+    const int seg_end = ROUTED ? a.tile_off[e] * 128 + a.counts[e] : rows;
 
     // A rows and B matrices of this block.
     const float *Bm0, *Bm1 = nullptr;
@@ -73,8 +75,7 @@ __global__ void __launch_bounds__(256) simt_expert_kernel(const SimtArgs a) {
             float av = 0.f;
             if (gr < rows && gk < K) {
                 if (MODE == SIMT_GATEUP_R) {
-                    const int tok = a.perm_tok[gr];
-                    av = tok >= 0 ? a.x[(size_t)tok * a.D + gk] : 0.f;
+                    av = gr < seg_end ? a.x[(size_t)a.perm_tok[gr] * a.D + gk] : 0.f;
                 } else if (MODE == SIMT_GATEUP_S) {
                     av = a.x[(size_t)gr * a.D + gk];
                 } else if (MODE == SIMT_DOWN_R) {
@@ -121,7 +122,7 @@ __global__ void __launch_bounds__(256) simt_expert_kernel(const SimtArgs a) {
             } else if (MODE == SIMT_GATEUP_S) {
                 a.h_sh[(size_t)r * a.d_sh + c] = silu_f(g[i][j]) * u[i][j];
             } else if (MODE == SIMT_DOWN_R) {
-                a.slot[(size_t)r * a.D + c] = a.w_perm[r] * g[i][j];
+                if (r < seg_end) a.slot[(size_t)r * a.D + c] = a.w_perm[r] * g[i][j];
             } else {
                 a.y[(size_t)r * a.D + c] = g[i][j];
             }
