@@ -3,10 +3,10 @@
 // sentinel of the GLM-5 experts' forward and goes nowhere).
 //
 // The N*k (token, slot) pairs are sorted by (expert, token, slot) into
-// expert-contiguous segments, each padded to a multiple of 128 rows so every
-// 128-row tile of the permuted layout belongs to one expert:
+// expert-contiguous segments, each padded to a multiple of the tile height (128
+// rows, or 32 for the decode kernels) so every tile belongs to one expert:
 //   1. count:   per-chunk expert histograms (shared-memory atomics)
-//   2. scan:    per-expert totals, per-chunk bases, 128-row tile prefix
+//   2. scan:    per-expert totals, per-chunk bases, tile prefix
 //   3. scatter: stable positions (warp match + per-warp counts), inverse map,
 //               per-row token id and routing weight
 //   4. gather:  copy each token's row of x to its permuted rows (bf16 path)
@@ -25,9 +25,10 @@ struct DispatchParams {
     const int32_t *topk_idx; // [N*k]
     const float *topk_w;     // [N*k]
     int N, k, E, nchunks;
+    int tile_rows;       // rows per tile of the permuted layout (128, or 32 for decode)
     int32_t *chunk_hist; // [nchunks][E] counts, then absolute bases
     int32_t *counts;     // [E]
-    int32_t *tile_off;   // [E+1] prefix of 128-row tiles per expert
+    int32_t *tile_off;   // [E+1] prefix of tiles per expert
     int32_t *meta;       // [0] done counter, [1] padded rows, [2] routed m-tiles
     int32_t *pos_of;     // [N*k] permuted row of each (token, slot), -1 if none
     int32_t *perm_tok;   // [rows_max] token of each permuted row (padding rows: unset)
@@ -67,7 +68,7 @@ __global__ void __launch_bounds__(DISPATCH_MAXE) dispatch_scan_kernel(const Disp
         }
         p.counts[e] = total;
     }
-    const int tiles = (e < p.E) ? (total + TILE_M - 1) / TILE_M : 0;
+    const int tiles = (e < p.E) ? (total + p.tile_rows - 1) / p.tile_rows : 0;
     // Block-wide exclusive scan of tiles.
     int v = tiles;
 #pragma unroll
@@ -91,13 +92,13 @@ __global__ void __launch_bounds__(DISPATCH_MAXE) dispatch_scan_kernel(const Disp
     const int excl = incl - tiles;
     if (e < p.E) {
         p.tile_off[e] = excl;
-        const int row0 = excl * TILE_M;
+        const int row0 = excl * p.tile_rows;
         for (int c = 0; c < p.nchunks; ++c) p.chunk_hist[(size_t)c * p.E + e] += row0;
     }
     if (e == p.E - 1) {
         p.tile_off[p.E] = incl;
         p.meta[0] = 0;
-        p.meta[1] = incl * TILE_M;
+        p.meta[1] = incl * p.tile_rows;
         p.meta[2] = incl;
     }
 }
@@ -153,7 +154,7 @@ __global__ void __launch_bounds__(DISPATCH_THREADS) dispatch_scatter_kernel(cons
     }
 }
 
-// Padding rows (beyond an expert's count inside its last 128-row tile) carry no
+// Padding rows (beyond an expert's count inside its last tile) carry no
 // token; perm_tok / w_perm are left unset there and every reader checks this.
 __device__ __forceinline__ int expert_of_tile(const int *tile_off, int E, int mt) {
     int lo = 0, hi = E - 1;
@@ -177,12 +178,12 @@ __global__ void __launch_bounds__(256) dispatch_gather_kernel(const uint8_t *__r
         if (e < p.E) s_cnt[e] = p.counts[e];
     }
     __syncthreads();
-    const int rows = min(s_off[p.E] * TILE_M, rows_max);
+    const int rows = min(s_off[p.E] * p.tile_rows, rows_max);
     const int lane = threadIdx.x & 31;
     for (int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < rows;
          r += (gridDim.x * blockDim.x) >> 5) {
-        const int e = expert_of_tile(s_off, p.E, r / TILE_M);
-        if (r - s_off[e] * TILE_M >= s_cnt[e]) continue; // padding row
+        const int e = expert_of_tile(s_off, p.E, r / p.tile_rows);
+        if (r - s_off[e] * p.tile_rows >= s_cnt[e]) continue; // padding row
         const int tok = p.perm_tok[r];
         const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)tok * row_bytes);
         uint4 *dst = reinterpret_cast<uint4 *>(x_perm + (size_t)r * row_bytes);

@@ -9,6 +9,7 @@
 #include "../../include/moe.h"
 #include "common.cuh"
 #include "dispatch.cuh"
+#include "gemm_decode_sm100.cuh"
 #include "gemm_sm100.cuh"
 #include "router.cuh"
 #include "simt_f32.cuh"
@@ -17,6 +18,9 @@ namespace moe {
 namespace {
 
 constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;
+// bf16 layers with at most this many tokens take the decode kernels (weights as
+// the 128-row MMA operand, 32-token tiles); larger ones the 128-row token tiles.
+constexpr int kDecodeMaxTokens = 256;
 uint64_t g_wait_limit_ns = kDefaultWaitLimitNs;
 int g_never_signal = 0;
 
@@ -43,7 +47,7 @@ struct DeviceInfo {
     int sms;
     int major, minor;
     bool gemm_attr_set;
-    bool router_attr_set;
+    bool dec_attr_set;
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -87,6 +91,8 @@ struct WsLayout {
     size_t x_perm, h_perm, h_sh, slot, total;
     int nchunks;
     size_t rows_max;
+    bool decode;
+    int tile_rows;
 };
 
 bool plan_workspace(int N, int D, int E, int d, int d_sh, int k, int dtype, WsLayout &L) {
@@ -95,7 +101,11 @@ bool plan_workspace(int N, int D, int E, int d, int d_sh, int k, int dtype, WsLa
     const size_t es = dtype == MOE_BF16 ? 2 : 4;
     const size_t nk = (size_t)N * (size_t)k;
     if (nk > (size_t)INT32_MAX / 2) return false;
-    L.rows_max = round_up(nk + (size_t)(TILE_M - 1) * E, TILE_M);
+    L.decode = dtype == MOE_BF16 && N <= kDecodeMaxTokens;
+    L.tile_rows = L.decode ? DEC_TT : TILE_M;
+    // Every non-empty expert pads its segment by at most tile_rows - 1 rows.
+    const size_t busy = std::min<size_t>((size_t)E, std::max<size_t>(nk, 1));
+    L.rows_max = round_up(nk + (size_t)(L.tile_rows - 1) * busy, TILE_M);
     if (L.rows_max > (size_t)INT32_MAX / 2) return false;
     L.nchunks = (int)((nk + DISPATCH_CHUNK - 1) / DISPATCH_CHUNK);
     size_t off = 0;
@@ -218,6 +228,40 @@ int launch_gemm(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap 
         cudaSuccess)
         return MOE_ERR_CUDA;
     return launch_status();
+}
+
+template <int KIND>
+int launch_decode(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &a2,
+                  const CUtensorMap &a3, const CUtensorMap &a4, const DecArgs &args, int grid,
+                  bool cooperative, cudaStream_t st) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(DEC_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = DEC_SMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = cooperative ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, grouped_gemm_decode_kernel<KIND>, a0, a1, a2, a3, a4, args) !=
+        cudaSuccess)
+        return MOE_ERR_CUDA;
+    return launch_status();
+}
+
+int ensure_decode_attrs(DeviceInfo *dev) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (dev->dec_attr_set) return MOE_OK;
+    if (cudaFuncSetAttribute(grouped_gemm_decode_kernel<GEMM_GATE_UP>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             DEC_SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(grouped_gemm_decode_kernel<GEMM_DOWN>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             DEC_SMEM_BYTES) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    dev->dec_attr_set = true;
+    return MOE_OK;
 }
 
 int ensure_gemm_attrs(DeviceInfo *dev) {
@@ -354,6 +398,7 @@ int moe_forward(const void *x, const void *gate_up, const void *down, const void
     dp.k = k;
     dp.E = E;
     dp.nchunks = L.nchunks;
+    dp.tile_rows = L.tile_rows;
     dp.chunk_hist = reinterpret_cast<int32_t *>(ws + L.chunk_hist);
     dp.counts = reinterpret_cast<int32_t *>(ws + L.counts);
     dp.tile_off = reinterpret_cast<int32_t *>(ws + L.tile_off);
@@ -418,11 +463,70 @@ int moe_forward(const void *x, const void *gate_up, const void *down, const void
                                                     D * 2, rows);
         if ((rc = launched(prof)) != MOE_OK) return rc;
     }
-    if ((rc = ensure_gemm_attrs(dev)) != MOE_OK) return rc;
     __nv_bfloat16 *h_perm = reinterpret_cast<__nv_bfloat16 *>(ws + L.h_perm);
     __nv_bfloat16 *h_sh = reinterpret_cast<__nv_bfloat16 *>(ws + L.h_sh);
     __nv_bfloat16 *slot = reinterpret_cast<__nv_bfloat16 *>(ws + L.slot);
 
+    if (L.decode) {
+        if ((rc = ensure_decode_attrs(dev)) != MOE_OK) return rc;
+        CUtensorMap mgu, mx_perm, msg, msu, mx, mdn, mh_perm, msd, mh_sh;
+        const bool ok =
+            make_map(&mgu, gate_up, D, (uint64_t)E * 2 * d_moe, D, 64) &&
+            make_map(&mx_perm, x_perm, D, L.rows_max, D, DEC_TT) &&
+            make_map(&msg, sh_gate, D, d_sh, D, 64) && make_map(&msu, sh_up, D, d_sh, D, 64) &&
+            make_map(&mx, x, D, N, D, DEC_TT) &&
+            make_map(&mdn, down, d_moe, (uint64_t)E * D, d_moe, DEC_BM) &&
+            make_map(&mh_perm, h_perm, d_moe, L.rows_max, d_moe, DEC_TT) &&
+            make_map(&msd, sh_down, d_sh, D, d_sh, DEC_BM) &&
+            make_map(&mh_sh, h_sh, d_sh, N, d_sh, DEC_TT);
+        if (!ok) return MOE_ERR_CUDA;
+        const int tt_max = (int)(L.rows_max / DEC_TT);
+        DecArgs g = {};
+        g.tile_off = dp.tile_off;
+        g.counts = dp.counts;
+        g.meta = dp.meta;
+        g.E = E;
+        g.N = N;
+        g.k = k;
+        g.tt_s = (N + DEC_TT - 1) / DEC_TT;
+        g.wait_limit_ns = g_wait_limit_ns;
+        g.never_signal = g_never_signal;
+        // gate_up + SwiGLU: 64 features x 32 tokens per tile
+        g.nb_r = (d_moe + 63) / 64;
+        g.nb_s = (d_sh + 63) / 64;
+        g.kb_r = g.kb_s = (D + DEC_BK - 1) / DEC_BK;
+        g.a_rows_per_e = 2 * d_moe;
+        g.up_off = d_moe;
+        g.out_r = h_perm;
+        g.ld_r = g.ncols_r = d_moe;
+        g.out_s = h_sh;
+        g.ld_s = g.ncols_s = d_sh;
+        int max_tiles = tt_max * g.nb_r + g.tt_s * g.nb_s;
+        rc = launch_decode<GEMM_GATE_UP>(mgu, mx_perm, msg, msu, mx, g,
+                                         std::min(dev->sms, max_tiles), false, st);
+        prof.mark();
+        if (rc != MOE_OK) return rc;
+        // down + weighted slot partials + shared expert + combine: 128 features x 32 tokens
+        g.nb_r = g.nb_s = (D + DEC_BM - 1) / DEC_BM;
+        g.kb_r = (d_moe + DEC_BK - 1) / DEC_BK;
+        g.kb_s = (d_sh + DEC_BK - 1) / DEC_BK;
+        g.a_rows_per_e = D;
+        g.up_off = 0;
+        g.out_r = slot;
+        g.ld_r = g.ncols_r = D;
+        g.out_s = static_cast<__nv_bfloat16 *>(y);
+        g.ld_s = g.ncols_s = D;
+        g.w_perm = dp.w_perm;
+        g.pos_of = dp.pos_of;
+        g.slot = slot;
+        max_tiles = tt_max * g.nb_r + g.tt_s * g.nb_s;
+        rc = launch_decode<GEMM_DOWN>(mdn, mh_perm, msd, msd, mh_sh, g,
+                                      std::min(dev->sms, max_tiles), true, st);
+        prof.mark();
+        return rc;
+    }
+
+    if ((rc = ensure_gemm_attrs(dev)) != MOE_OK) return rc;
     CUtensorMap mx_perm, mgu, mx, msg, msu, mh_perm, mdn, mh_sh, msd;
     bool ok = make_map(&mx_perm, x_perm, D, L.rows_max, D, 128) &&
               make_map(&mgu, gate_up, D, (uint64_t)E * 2 * d_moe, D, 128) &&

@@ -109,6 +109,11 @@ SMALL = {
                                         d_moe=128, d_sh=256, skew=False)),
     "bf16_single_token": ("glm5_decode", dict(N=1, D=256, E=16, k=8, d_moe=128, d_sh=128)),
     "bf16_k1_e1": ("glm5_decode", dict(N=130, D=128, E=1, k=1, d_moe=64, d_sh=64)),
+    # N <= 256 takes the decode kernels (weights as the 128-row MMA operand, 32-token tiles)
+    "bf16_decode_ragged": ("glm5_decode", dict(N=100, D=520, E=6, k=3, d_moe=200, d_sh=136)),
+    "bf16_decode_multitile": ("glm5_decode", dict(N=250, D=256, E=4, k=2, d_moe=128, d_sh=64)),
+    "bf16_decode_group": ("skew_grouped", dict(N=64, D=384, E=64, n_group=8, topk_group=4, k=8,
+                                               d_moe=192, d_sh=320, skew=False)),
     "fp32_tiny": ("tiny_fp32", dict()),
     "fp32_ragged": ("tiny_fp32", dict(N=77, D=100, E=6, n_group=2, topk_group=1, k=2,
                                       d_moe=40, d_sh=24)),
@@ -139,8 +144,9 @@ def test_forward_parity_small(case):
     assert err2["max_rel"] <= Y_TOL[cfg.dtype]
 
 
-def test_forward_sentinel_and_hot_expert():
-    cfg = CONFIGS["glm5_prefill"].with_(N=400, D=256, E=8, k=4, d_moe=128, d_sh=128)
+@pytest.mark.parametrize("N", [200, 400])
+def test_forward_sentinel_and_hot_expert(N):
+    cfg = CONFIGS["glm5_prefill"].with_(N=N, D=256, E=8, k=4, d_moe=128, d_sh=128)
     inp = make_inputs(cfg, seed=2)
     rng = np.random.default_rng(3)
     idx = np.stack([rng.permutation(cfg.E)[:cfg.k] for _ in range(cfg.N)]).astype(np.int32)
@@ -165,8 +171,9 @@ def test_forward_zero_tokens_is_noop():
     assert moe.moe_device_status() == 0
 
 
-def test_forward_is_deterministic():
-    cfg = CONFIGS["glm5_prefill"].with_(N=1000, D=512, E=16, k=8, d_moe=256, d_sh=256)
+@pytest.mark.parametrize("N", [100, 1000])
+def test_forward_is_deterministic(N):
+    cfg = CONFIGS["glm5_prefill"].with_(N=N, D=512, E=16, k=8, d_moe=256, d_sh=256)
     inp = make_inputs(cfg, seed=4, device=DEV)
     y1, _, _ = moe.moe_layer(inp.x, inp.W_g, inp.b, *_weights(inp)[1:], 1, 1, 8, True, 2.5)
     y2, _, _ = moe.moe_layer(inp.x, inp.W_g, inp.b, *_weights(inp)[1:], 1, 1, 8, True, 2.5)
@@ -191,8 +198,9 @@ def test_bad_expert_id_is_skipped_and_reported():
     assert moe.moe_device_status() == 0  # cleared
 
 
-def test_bounded_wait_times_out_and_context_survives():
-    cfg = CONFIGS["glm5_prefill"].with_(N=256, D=256, E=8, k=2, d_moe=128, d_sh=128)
+@pytest.mark.parametrize("N", [256, 600])
+def test_bounded_wait_times_out_and_context_survives(N):
+    cfg = CONFIGS["glm5_prefill"].with_(N=N, D=256, E=8, k=2, d_moe=128, d_sh=128)
     inp = make_inputs(cfg, seed=8, device=DEV)
     idx, w = moe.moe_router(inp.x, inp.W_g, inp.b, 1, 1, 2, True, 2.5)
     moe.moe_debug_set_wait_limit_ns(20_000_000)
