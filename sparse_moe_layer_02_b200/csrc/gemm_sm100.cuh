@@ -20,11 +20,13 @@
 // the routed tiles in the same launch.
 //
 // down: one tile = 128 rows x 256 output columns of W_down (D x d_moe).  Routed
-// tiles scale each row by its routing weight and store a bf16 per-slot partial.
-// The shared expert's tiles come last: after a bounded wait until every routed
-// tile is stored, each row n adds its k slot partials in slot order and the
-// shared expert's fp32 accumulator (scale 1), and writes y once in bf16
-// (deterministic: no atomics on the output).
+// tiles scale each row by its routing weight and store a bf16 per-slot partial;
+// the shared expert's tiles store their fp32 output.  Every tile then bumps a
+// done counter.  When a CTA has no tiles left it waits (bounded) for the counter
+// to cover every tile of the launch, and then all CTAs of the same persistent
+// launch combine: row n of y = the k slot partials summed in slot order plus the
+// shared expert's output at scale 1, written once in bf16 (deterministic: no
+// atomics on the output), one warp per row with 16-byte loads.
 #pragma once
 
 #include "common.cuh"
@@ -64,6 +66,7 @@ struct GemmArgs {
     const float *w_perm;   // down: routing weight per permuted row
     const int32_t *pos_of; // down: [N*k] permuted row of (n, j), -1 if none
     const __nv_bfloat16 *slot; // down: slot partials (same as out_r)
+    float *osh;                // down: shared expert output [N, ld_s] fp32
     uint64_t wait_limit_ns;
     int never_signal;
 };
@@ -120,6 +123,54 @@ __device__ __forceinline__ void store_row_chunk_bf16(__nv_bfloat16 *row_ptr, int
 #pragma unroll
     for (int q = 0; q < 4; ++q)
         if (col + 8 * q < ncols) dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+}
+
+// y[n] = sum_{j<k} slot[pos(n, j)] (slot order) + osh[n], one warp per row, each
+// lane two 8-column pieces at a time so 2(k+2) 16-byte loads are in flight.
+__device__ __forceinline__ void combine_rows(const GemmArgs &a, int gwarp, int nwarps, int lane) {
+    const int pieces = a.ncols_s / 8;
+    for (int n = gwarp; n < a.N; n += nwarps) {
+        const int my_pos = lane < a.k ? a.pos_of[(size_t)n * a.k + lane] : -1;
+        // Uniform trip count across the warp: the shuffles below need every lane.
+        for (int pbase = 0; pbase < pieces; pbase += 64) {
+            const int p0 = pbase + lane;
+            float sum[2][8];
+#pragma unroll
+            for (int u = 0; u < 2; ++u)
+#pragma unroll
+                for (int h = 0; h < 8; ++h) sum[u][h] = 0.f;
+            for (int j = 0; j < a.k; ++j) {
+                const int p = __shfl_sync(0xffffffffu, my_pos, j);
+                if (p < 0) continue;
+                const __nv_bfloat16 *srow = a.slot + (size_t)p * a.ld_r;
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int pc = p0 + 32 * u;
+                    if (pc < pieces) {
+                        const uint4 w4 = __ldcg(reinterpret_cast<const uint4 *>(srow + pc * 8));
+                        float lo, hi;
+                        unpack_bf16x2(w4.x, lo, hi); sum[u][0] += lo; sum[u][1] += hi;
+                        unpack_bf16x2(w4.y, lo, hi); sum[u][2] += lo; sum[u][3] += hi;
+                        unpack_bf16x2(w4.z, lo, hi); sum[u][4] += lo; sum[u][5] += hi;
+                        unpack_bf16x2(w4.w, lo, hi); sum[u][6] += lo; sum[u][7] += hi;
+                    }
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int pc = p0 + 32 * u;
+                if (pc < pieces) {
+                    const float4 *o = reinterpret_cast<const float4 *>(a.osh + (size_t)n * a.ld_s + pc * 8);
+                    const float4 o0 = __ldcg(o), o1 = __ldcg(o + 1);
+                    const uint4 out = make_uint4(pack_bf16x2(sum[u][0] + o0.x, sum[u][1] + o0.y),
+                                                 pack_bf16x2(sum[u][2] + o0.z, sum[u][3] + o0.w),
+                                                 pack_bf16x2(sum[u][4] + o1.x, sum[u][5] + o1.y),
+                                                 pack_bf16x2(sum[u][6] + o1.z, sum[u][7] + o1.w));
+                    *reinterpret_cast<uint4 *>(a.out_s + (size_t)n * a.ld_s + pc * 8) = out;
+                }
+            }
+        }
+    }
 }
 
 template <int KIND>
@@ -264,24 +315,6 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++tc) {
             const TileCoord c = decode_tile(t, routed_tiles, a, s_tile_off);
             const uint32_t acc = tc & 1, aph = (tc >> 1) & 1;
-            bool do_combine = true;
-            if (KIND == GEMM_DOWN && c.shared) {
-                // Wait until every routed tile has stored its slot partials.
-                if (ep_tid == 0 && !*combine_failed && !*abort_flag) {
-                    const int target = routed_tiles + (a.never_signal ? 1 : 0);
-                    const uint64_t t0 = globaltimer_ns();
-                    while (ld_acquire_gpu(&a.meta[0]) < target) {
-                        if (globaltimer_ns() - t0 > limit) {
-                            record_error(DEV_TIMEOUT, 120);
-                            *combine_failed = 1;
-                            break;
-                        }
-                        __nanosleep(200);
-                    }
-                }
-                named_bar_sync(1, 128);
-                do_combine = !*combine_failed;
-            }
             // After an abort every wait fails at once; the loop still walks the same
             // tiles in every epilogue warp so the named barriers stay matched.
             // One lane waits; the result is made warp-uniform before the
@@ -334,39 +367,22 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     }
                 }
             } else {
+                // shared expert: fp32 output rows, combined after every tile is done
                 const int n = c.a_row + row;
-                const bool row_ok = n < a.N && do_combine;
-                __nv_bfloat16 *row_ptr = a.out_s + (size_t)n * a.ld_s;
+                float *row_ptr = a.osh + (size_t)n * a.ld_s;
 #pragma unroll 1
                 for (int ch = 0; ch < 8; ++ch) {
                     uint32_t v[32];
                     tmem_ld_32x32b_x32(tbase + ch * 32, v);
                     tmem_ld_wait();
                     const int col = c.nb * GEMM_BN + ch * 32;
-                    if (row_ok && col < a.ncols_s) {
-                        float sum[32];
+                    if (n < a.N && col < a.ncols_s) {
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) sum[i] = 0.f;
-                        for (int j = 0; j < a.k; ++j) {
-                            const int p = a.pos_of[(size_t)n * a.k + j];
-                            if (p < 0) continue;
-                            const uint4 *src =
-                                reinterpret_cast<const uint4 *>(a.slot + (size_t)p * a.ld_r + col);
-#pragma unroll
-                            for (int qv = 0; qv < 4; ++qv) {
-                                if (col + 8 * qv < a.ncols_s) {
-                                    const uint4 w4 = __ldcg(src + qv);
-                                    float lo, hi;
-                                    unpack_bf16x2(w4.x, lo, hi); sum[8 * qv + 0] += lo; sum[8 * qv + 1] += hi;
-                                    unpack_bf16x2(w4.y, lo, hi); sum[8 * qv + 2] += lo; sum[8 * qv + 3] += hi;
-                                    unpack_bf16x2(w4.z, lo, hi); sum[8 * qv + 4] += lo; sum[8 * qv + 5] += hi;
-                                    unpack_bf16x2(w4.w, lo, hi); sum[8 * qv + 6] += lo; sum[8 * qv + 7] += hi;
-                                }
-                            }
-                        }
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) sum[i] += __uint_as_float(v[i]);
-                        store_row_chunk_bf16(row_ptr, col, a.ncols_s, sum);
+                        for (int qv = 0; qv < 8; ++qv)
+                            if (col + 4 * qv < a.ncols_s)
+                                reinterpret_cast<float4 *>(row_ptr + col)[qv] =
+                                    make_float4(__uint_as_float(v[4 * qv]), __uint_as_float(v[4 * qv + 1]),
+                                                __uint_as_float(v[4 * qv + 2]), __uint_as_float(v[4 * qv + 3]));
                     }
                 }
             }
@@ -375,8 +391,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty[acc]);
             }  // have
-            if (KIND == GEMM_DOWN && !c.shared) {
-                // Publish this routed tile's partials to the shared-expert tiles.
+            if (KIND == GEMM_DOWN) {
+                // Publish this tile's stores to the combine phase.
                 __threadfence();
                 named_bar_sync(1, 128);
                 if (ep_tid == 0 && have) atomicAdd(&a.meta[0], 1);
@@ -389,6 +405,25 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, GEMM_TMEM_COLS);
+    }
+
+    if (KIND == GEMM_DOWN) {
+        // ---- combine phase: every tile of the launch must be stored first ----------
+        if (threadIdx.x == 0 && !*abort_flag) {
+            const int target = total_tiles + (a.never_signal ? 1 : 0);
+            const uint64_t t0 = globaltimer_ns();
+            while (ld_acquire_gpu(&a.meta[0]) < target) {
+                if (globaltimer_ns() - t0 > limit) {
+                    record_error(DEV_TIMEOUT, 120);
+                    *combine_failed = 1;
+                    break;
+                }
+                __nanosleep(256);
+            }
+        }
+        __syncthreads();
+        if (!*combine_failed && !*abort_flag) combine_rows(a, blockIdx.x * (GEMM_THREADS / 32) + warp,
+                                                           gridDim.x * (GEMM_THREADS / 32), lane);
     }
 }
 

@@ -12,6 +12,7 @@
 #include "gemm_decode_sm100.cuh"
 #include "gemm_sm100.cuh"
 #include "router.cuh"
+#include "router_tc.cuh"
 #include "simt_f32.cuh"
 
 namespace moe {
@@ -88,7 +89,7 @@ int check_router_shape(int N, int D, int E, int G, int tg, int k) {
 // ---------------------------------------------------------------------------
 struct WsLayout {
     size_t chunk_hist, counts, tile_off, meta, pos_of, perm_tok, w_perm;
-    size_t x_perm, h_perm, h_sh, slot, total;
+    size_t x_perm, h_perm, h_sh, slot, osh, total;
     int nchunks;
     size_t rows_max;
     bool decode;
@@ -125,6 +126,8 @@ bool plan_workspace(int N, int D, int E, int d, int d_sh, int k, int dtype, WsLa
     L.h_perm = take(L.rows_max * d * es);
     L.h_sh = take((size_t)N * d_sh * es);
     L.slot = take(L.rows_max * D * es);
+    // fp32 output of the shared expert, combined with the slots (prefill kernels)
+    L.osh = take(dtype == MOE_BF16 && !L.decode ? (size_t)N * D * 4 : 0);
     L.total = off;
     return true;
 }
@@ -208,6 +211,49 @@ int launch_router_x(const RouterParams &p, cudaStream_t st) {
     if (p.E <= 128) return launch_router_t<XT, WT, 4>(p, st);
     if (p.E <= 256) return launch_router_t<XT, WT, 8>(p, st);
     return launch_router_t<XT, WT, 16>(p, st);
+}
+
+template <int EV>
+int launch_router_tc_t(const CUtensorMap &mX, const CUtensorMap &mW, const RouterParams &p, int clk,
+                       cudaStream_t st) {
+    static bool attr_set = false;
+    if (!attr_set) {
+        if (cudaFuncSetAttribute(router_tc_kernel<EV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 RTC_SMEM_BYTES) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        attr_set = true;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(clk, (p.N + RTC_BM - 1) / RTC_BM, 1);
+    cfg.blockDim = dim3(RTC_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = RTC_SMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = clk;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, router_tc_kernel<EV>, mX, mW, p, g_wait_limit_ns) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    return launch_status();
+}
+
+// Tensor-core router for bf16 x and bf16 W_g with 16 <= E <= 256, E % 16 == 0.
+int launch_router_tc(const RouterParams &p, int sms, cudaStream_t st) {
+    CUtensorMap mX, mW;
+    if (!make_map(&mX, p.x, p.D, p.N, p.D, RTC_BM) || !make_map(&mW, p.W_g, p.D, p.E, p.D, p.E))
+        return MOE_ERR_CUDA;
+    const int tblocks = (p.N + RTC_BM - 1) / RTC_BM;
+    // K-split cluster size: a power of two (so it divides the 128 tokens of a
+    // block) chosen to put about one CTA on every SM, at most 8.
+    int clk = 1;
+    while (clk < 8 && 2 * clk * tblocks <= sms) clk *= 2;
+    if (p.E <= 32) return launch_router_tc_t<1>(mX, mW, p, clk, st);
+    if (p.E <= 64) return launch_router_tc_t<2>(mX, mW, p, clk, st);
+    if (p.E <= 128) return launch_router_tc_t<4>(mX, mW, p, clk, st);
+    return launch_router_tc_t<8>(mX, mW, p, clk, st);
 }
 
 template <int KIND>
@@ -351,6 +397,9 @@ int moe_router(const void *x, int x_dtype, const void *W_g, int wg_dtype, const 
     p.topk_idx = topk_idx;
     p.topk_w = topk_w;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (x_dtype == MOE_BF16 && wg_dtype == MOE_BF16 && E % 16 == 0 && E >= 16 && E <= 256 &&
+        D % 8 == 0)
+        return launch_router_tc(p, dev->sms, st);
     if (x_dtype == MOE_F32 && wg_dtype == MOE_F32) return launch_router_x<float, float>(p, st);
     if (x_dtype == MOE_BF16 && wg_dtype == MOE_F32) return launch_router_x<__nv_bfloat16, float>(p, st);
     if (x_dtype == MOE_BF16 && wg_dtype == MOE_BF16)
@@ -583,6 +632,7 @@ int moe_forward(const void *x, const void *gate_up, const void *down, const void
     g.w_perm = dp.w_perm;
     g.pos_of = dp.pos_of;
     g.slot = slot;
+    g.osh = reinterpret_cast<float *>(ws + L.osh);
     max_tiles = mt_r_max * g.nb_r + mt_s * g.nb_s;
     rc = launch_gemm<GEMM_DOWN>(mh_perm, mdn, mh_sh, msd, msd, g, std::min(dev->sms, max_tiles),
                                 true, st);

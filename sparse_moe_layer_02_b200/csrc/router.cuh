@@ -61,6 +61,120 @@ __device__ __forceinline__ void warp_argmax(float &v, int &i) {
     }
 }
 
+// Selection for one token by one warp ("GLM-4.5 Group Router", How it works):
+// lane l holds the fp32 logits of experts l, l+32, ...  s = sigmoid(r),
+// s' = s + b; with n_group > 1 a group scores the sum of its two largest s' and
+// the topk_group best groups are kept (others are -inf); the k largest s' among
+// the kept experts are chosen (ties to the lower id) and their weights are
+// alpha * s / (sum of the chosen s + 1e-20), or alpha * s without normalisation.
+// sp_w is a per-warp scratch row of 32 * ROUTER_MAXV floats in shared memory.
+template <int EV>
+__device__ __forceinline__ void router_select(const RouterParams &p, int t, const float (&logit)[EV],
+                                              float *sp_w, int lane) {
+    const int E = p.E, G = p.G, m = E / G;
+    float s[EV], sp[EV];
+#pragma unroll
+    for (int v = 0; v < EV; ++v) {
+        const int e = lane + 32 * v;
+        s[v] = 0.f;
+        sp[v] = -INFINITY;
+        if (e < E) {
+            s[v] = 1.0f / (1.0f + expf(-logit[v]));
+            sp[v] = s[v] + p.b[e];
+        }
+    }
+    // Candidate mask over this lane's experts (bit v).
+    uint32_t cand = 0;
+    if (G > 1) {
+#pragma unroll
+        for (int v = 0; v < EV; ++v)
+            if (lane + 32 * v < E) sp_w[lane + 32 * v] = sp[v];
+        __syncwarp();
+        // Group score = sum of the two largest s' of the group (lanes own g, g+32).
+        float gs[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int g = lane + 32 * h;
+            if (g < G) {
+                float b1 = -INFINITY, b2 = -INFINITY;
+                for (int q = g * m; q < (g + 1) * m; ++q) {
+                    const float v = sp_w[q];
+                    if (v > b1) {
+                        b2 = b1;
+                        b1 = v;
+                    } else if (v > b2) {
+                        b2 = v;
+                    }
+                }
+                gs[h] = b1 + b2;
+            }
+        }
+        __syncwarp();
+        uint64_t kept = 0;
+        for (int r = 0; r < p.tg; ++r) {
+            float bv = -INFINITY;
+            int bi = 0x7fffffff;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int g = lane + 32 * h;
+                if (g < G && !((kept >> g) & 1ull) && better(gs[h], g, bv, bi)) {
+                    bv = gs[h];
+                    bi = g;
+                }
+            }
+            warp_argmax(bv, bi);
+            kept |= 1ull << bi;
+        }
+#pragma unroll
+        for (int v = 0; v < EV; ++v) {
+            const int e = lane + 32 * v;
+            if (e < E && ((kept >> (e / m)) & 1ull)) cand |= 1u << v;
+        }
+    } else {
+#pragma unroll
+        for (int v = 0; v < EV; ++v)
+            if (lane + 32 * v < E) cand |= 1u << v;
+    }
+    // Top-k by s' among candidates; lane r keeps the r-th pick.
+    int my_e = -1;
+    float my_s = 0.f;
+    for (int r = 0; r < p.k; ++r) {
+        float bv = -INFINITY;
+        int bi = 0x7fffffff;
+#pragma unroll
+        for (int v = 0; v < EV; ++v) {
+            if ((cand >> v) & 1u) {
+                const int e = lane + 32 * v;
+                if (better(sp[v], e, bv, bi)) {
+                    bv = sp[v];
+                    bi = e;
+                }
+            }
+        }
+        warp_argmax(bv, bi);
+        const int owner = bi & 31, vw = bi >> 5;
+        float sv = 0.f;
+#pragma unroll
+        for (int v = 0; v < EV; ++v)
+            if (v == vw) sv = s[v];
+        sv = __shfl_sync(0xffffffffu, sv, owner);
+        if (lane == owner) cand &= ~(1u << vw);
+        if (lane == r) {
+            my_e = bi;
+            my_s = sv;
+        }
+    }
+    // Weights from the raw scores of the chosen set.
+    float sum = (lane < p.k) ? my_s : 0.f;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+    if (lane < p.k) {
+        const float w = p.norm ? p.alpha * my_s / (sum + 1e-20f) : p.alpha * my_s;
+        p.topk_idx[(size_t)t * p.k + lane] = my_e;
+        p.topk_w[(size_t)t * p.k + lane] = w;
+    }
+}
+
 // EV = experts per lane (E <= 32 * EV); each thread accumulates 4 tokens x EV experts.
 template <typename XT, typename WT, int EV>
 __global__ void __launch_bounds__(ROUTER_THREADS)
@@ -150,118 +264,24 @@ __global__ void __launch_bounds__(ROUTER_THREADS)
     cluster.sync();
 
     // ---- reduce over the cluster's K slices, then select: one warp per token ----
-    const int G = p.G, m = E / G;
     const int j = rank + ROUTER_CL * warp; // token of this warp (32 = CL * 4 tokens per cluster)
     const int t = t0 + j;
     if (warp < ROUTER_TM / ROUTER_CL && t < p.N) {
-        float *sp_w = spbuf + warp * ROUTER_MAXV * 32;
-        float s[EV], sp[EV];
+        float logit[EV];
 #pragma unroll
         for (int v = 0; v < EV; ++v) {
             const int e = lane + 32 * v;
-            s[v] = 0.f;
-            sp[v] = -INFINITY;
+            float r = 0.f;
             if (e < E) {
-                float r = 0.f;
 #pragma unroll
                 for (int c = 0; c < ROUTER_CL; ++c) {
                     const float *remote = cluster.map_shared_rank(part, c);
                     r += remote[j * EP + e];
                 }
-                s[v] = 1.0f / (1.0f + expf(-r));
-                sp[v] = s[v] + p.b[e];
             }
+            logit[v] = r;
         }
-        // Candidate mask over this lane's experts (bit v).
-        uint32_t cand = 0;
-        if (G > 1) {
-#pragma unroll
-            for (int v = 0; v < EV; ++v)
-                if (lane + 32 * v < E) sp_w[lane + 32 * v] = sp[v];
-            __syncwarp();
-            // Group score = sum of the two largest s' of the group (lanes own g, g+32).
-            float gs[2] = {-INFINITY, -INFINITY};
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int g = lane + 32 * h;
-                if (g < G) {
-                    float b1 = -INFINITY, b2 = -INFINITY;
-                    for (int q = g * m; q < (g + 1) * m; ++q) {
-                        const float v = sp_w[q];
-                        if (v > b1) {
-                            b2 = b1;
-                            b1 = v;
-                        } else if (v > b2) {
-                            b2 = v;
-                        }
-                    }
-                    gs[h] = b1 + b2;
-                }
-            }
-            __syncwarp();
-            uint64_t kept = 0;
-            for (int r = 0; r < p.tg; ++r) {
-                float bv = -INFINITY;
-                int bi = 0x7fffffff;
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int g = lane + 32 * h;
-                    if (g < G && !((kept >> g) & 1ull) && better(gs[h], g, bv, bi)) {
-                        bv = gs[h];
-                        bi = g;
-                    }
-                }
-                warp_argmax(bv, bi);
-                kept |= 1ull << bi;
-            }
-#pragma unroll
-            for (int v = 0; v < EV; ++v) {
-                const int e = lane + 32 * v;
-                if (e < E && ((kept >> (e / m)) & 1ull)) cand |= 1u << v;
-            }
-        } else {
-#pragma unroll
-            for (int v = 0; v < EV; ++v)
-                if (lane + 32 * v < E) cand |= 1u << v;
-        }
-        // Top-k by s' among candidates; lane r keeps the r-th pick.
-        int my_e = -1;
-        float my_s = 0.f;
-        for (int r = 0; r < p.k; ++r) {
-            float bv = -INFINITY;
-            int bi = 0x7fffffff;
-#pragma unroll
-            for (int v = 0; v < EV; ++v) {
-                if ((cand >> v) & 1u) {
-                    const int e = lane + 32 * v;
-                    if (better(sp[v], e, bv, bi)) {
-                        bv = sp[v];
-                        bi = e;
-                    }
-                }
-            }
-            warp_argmax(bv, bi);
-            const int owner = bi & 31, vw = bi >> 5;
-            float sv = 0.f;
-#pragma unroll
-            for (int v = 0; v < EV; ++v)
-                if (v == vw) sv = s[v];
-            sv = __shfl_sync(0xffffffffu, sv, owner);
-            if (lane == owner) cand &= ~(1u << vw);
-            if (lane == r) {
-                my_e = bi;
-                my_s = sv;
-            }
-        }
-        // Weights from the raw scores of the chosen set.
-        float sum = (lane < p.k) ? my_s : 0.f;
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-        if (lane < p.k) {
-            const float w = p.norm ? p.alpha * my_s / (sum + 1e-20f) : p.alpha * my_s;
-            p.topk_idx[(size_t)t * p.k + lane] = my_e;
-            p.topk_w[(size_t)t * p.k + lane] = w;
-        }
+        router_select<EV>(p, t, logit, spbuf + warp * ROUTER_MAXV * 32, lane);
     }
     cluster.sync(); // keep this CTA's partials alive until every reader is done
 }
