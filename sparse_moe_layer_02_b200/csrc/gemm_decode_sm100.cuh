@@ -178,7 +178,11 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
             for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
                 const DecTile c = dec_decode_tile(t, routed_tiles, a, s_off, s_cnt);
                 const CUtensorMap *mB = c.shared ? &mB_s : &mB_r;
-                for (int kb = 0; kb < c.kb; ++kb, ++it) {
+                // Feature blocks of one token tile run on neighbouring CTAs and share
+                // the token tile; start each at a different k-block.
+                const int rot = c.fb % c.kb;
+                for (int i = 0; i < c.kb; ++i, ++it) {
+                    const int kb = i + rot < c.kb ? i + rot : i + rot - c.kb;
                     const uint32_t s = it % DEC_STAGES, ph = (it / DEC_STAGES) & 1;
                     if (!mbar_wait(&empty[s], ph ^ 1, limit, abort_flag, 200)) { ok = false; break; }
                     uint8_t *sa = ring + s * DEC_STAGE_BYTES;
@@ -211,6 +215,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
                 }
             }
         }
+        __syncwarp(); // lanes 1-31 wait here for lane 0: the warp reconverges
     } else if (warp == 1) {
         // ------------------------------ MMA issuer --------------------------------
         if (lane == 0) {
@@ -223,7 +228,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
                 if (!mbar_wait(&tempty[acc], aph ^ 1, limit, abort_flag, 210)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + acc * DEC_TT;
-                for (int kb = 0; kb < c.kb; ++kb, ++it) {
+                for (int i = 0; i < c.kb; ++i, ++it) {
                     const uint32_t s = it % DEC_STAGES, ph = (it / DEC_STAGES) & 1;
                     if (!mbar_wait(&full[s], ph, limit, abort_flag, 211)) { ok = false; break; }
                     tc_fence_after();
@@ -233,7 +238,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
                     for (int kk = 0; kk < DEC_BK / 16; ++kk)
                         umma_bf16_ss(d_tmem, umma_desc_sw128(sa + kk * 32),
                                      umma_desc_sw128(sb + kk * 32), idesc,
-                                     (kb > 0 || kk > 0) ? 1u : 0u);
+                                     (i > 0 || kk > 0) ? 1u : 0u);
                     umma_commit(&empty[s]);
                 }
                 if (!ok) break;
@@ -243,6 +248,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
             volatile int no_abort = 0;
             mbar_wait(drain, 0, 100000000ull, &no_abort, 212);
         }
+        __syncwarp();
     } else {
         // ------------------------------ epilogue ---------------------------------
         const int q = warp & 3;

@@ -239,7 +239,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
                 const TileCoord c = decode_tile(t, routed_tiles, a, s_tile_off);
                 const CUtensorMap *mA = c.shared ? &mA_s : &mA_r;
-                for (int kb = 0; kb < c.kb; ++kb, ++it) {
+                // The n-blocks of one m-tile run on neighbouring CTAs and share the A
+                // tile; each starts at a different k-block so they do not all request
+                // the same lines at the same time.
+                const int rot = c.nb % c.kb;
+                for (int i = 0; i < c.kb; ++i, ++it) {
+                    const int kb = i + rot < c.kb ? i + rot : i + rot - c.kb;
                     const uint32_t s = it % GEMM_STAGES, ph = (it / GEMM_STAGES) & 1;
                     if (!mbar_wait(&empty[s], ph ^ 1, limit, abort_flag, 100)) { ok = false; break; }
                     uint8_t *sa = ring + s * GEMM_STAGE_BYTES;
@@ -273,6 +278,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 }
             }
         }
+        __syncwarp(); // lanes 1-31 wait here for lane 0: the warp reconverges
     } else if (warp == 1) {
         // ------------------------------ MMA issuer --------------------------------
         if (lane == 0) {
@@ -285,7 +291,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 if (!mbar_wait(&tempty[acc], aph ^ 1, limit, abort_flag, 110)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + acc * GEMM_BN;
-                for (int kb = 0; kb < c.kb; ++kb, ++it) {
+                for (int i = 0; i < c.kb; ++i, ++it) {
                     const uint32_t s = it % GEMM_STAGES, ph = (it / GEMM_STAGES) & 1;
                     if (!mbar_wait(&full[s], ph, limit, abort_flag, 111)) { ok = false; break; }
                     tc_fence_after();
@@ -295,7 +301,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     for (int kk = 0; kk < GEMM_BK / 16; ++kk)
                         umma_bf16_ss(d_tmem, umma_desc_sw128(sa + kk * 32),
                                      umma_desc_sw128(sb + kk * 32), idesc,
-                                     (kb > 0 || kk > 0) ? 1u : 0u);
+                                     (i > 0 || kk > 0) ? 1u : 0u);
                     umma_commit(&empty[s]);
                 }
                 if (!ok) break;
@@ -306,6 +312,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             volatile int no_abort = 0;
             mbar_wait(drain, 0, 100000000ull, &no_abort, 112);
         }
+        __syncwarp();
     } else {
         // ------------------------------ epilogue ---------------------------------
         const int q = warp & 3;          // TMEM lane quadrant of this warp

@@ -229,8 +229,16 @@ __global__ void __launch_bounds__(ROUTER_THREADS)
             wr[q] = (r < E && kk < kend) ? to_f32(W[(size_t)r * p.D + kk]) : 0.f;
         }
     };
-    if (kbeg < kend) load_chunk(kbeg);
-    for (int k0 = kbeg; k0 < kend; k0 += ROUTER_KC) {
+    // Clusters of different token blocks read the same W_g columns; rotating the
+    // chunk order by the token block keeps them on different L2 lines.
+    const int nch = kend > kbeg ? (kend - kbeg + ROUTER_KC - 1) / ROUTER_KC : 0;
+    const int rot = nch > 0 ? (int)(blockIdx.y % (unsigned)nch) : 0;
+    auto chunk_k0 = [&](int i) {
+        const int c = i + rot < nch ? i + rot : i + rot - nch;
+        return kbeg + c * ROUTER_KC;
+    };
+    if (nch > 0) load_chunk(chunk_k0(0));
+    for (int ci = 0; ci < nch; ++ci) {
 #pragma unroll
         for (int q = 0; q < XPT; ++q) {
             const int i = tid + ROUTER_THREADS * q;
@@ -242,7 +250,7 @@ __global__ void __launch_bounds__(ROUTER_THREADS)
             ws[i / ROUTER_KC][i % ROUTER_KC] = wr[q];
         }
         __syncthreads();
-        if (k0 + ROUTER_KC < kend) load_chunk(k0 + ROUTER_KC);
+        if (ci + 1 < nch) load_chunk(chunk_k0(ci + 1));
 #pragma unroll 4
         for (int kk = 0; kk < ROUTER_KC; ++kk) {
             float a[4], w[EV];

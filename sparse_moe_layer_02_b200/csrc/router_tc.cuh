@@ -58,6 +58,11 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
     const int kper = (KB + CLK - 1) / CLK;
     const int kb0 = rank * kper, kb1 = min(KB, kb0 + kper);
     const uint32_t b_bytes = (uint32_t)E * RTC_BK * 2;
+    // Every CTA reads the same W_g slices; rotating the k-block order by the token
+    // block spreads concurrent reads over different L2 lines instead of having all
+    // CTAs request the same 32 KiB at once.
+    const int nkb = kb1 - kb0;
+    const int rot = nkb > 0 ? (int)(blockIdx.y % (unsigned)nkb) : 0;
     const uint32_t tmem_cols = E <= 32 ? 32 : E <= 64 ? 64 : E <= 128 ? 128 : 256;
 
     if (threadIdx.x == 0) {
@@ -86,7 +91,8 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
         if (lane == 0) {
             uint32_t it = 0;
             bool ok = true;
-            for (int kb = kb0; kb < kb1; ++kb, ++it) {
+            for (int i = 0; i < nkb; ++i, ++it) {
+                const int kb = kb0 + (i + rot < nkb ? i + rot : i + rot - nkb);
                 const uint32_t s = it % RTC_STAGES, ph = (it / RTC_STAGES) & 1;
                 if (!mbar_wait(&empty[s], ph ^ 1, limit, abort_flag, 300)) { ok = false; break; }
                 uint8_t *sa = ring + s * RTC_STAGE_BYTES;
@@ -102,11 +108,12 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
                 }
             }
         }
+        __syncwarp(); // lanes 1-31 wait here for lane 0: the warp reconverges
     } else if (warp == 1) {
         if (lane == 0) {
             const uint32_t idesc = umma_idesc_bf16(RTC_BM, E);
             uint32_t it = 0;
-            for (int kb = kb0; kb < kb1; ++kb, ++it) {
+            for (int i = 0; i < nkb; ++i, ++it) {
                 const uint32_t s = it % RTC_STAGES, ph = (it / RTC_STAGES) & 1;
                 if (!mbar_wait(&full[s], ph, limit, abort_flag, 310)) break;
                 tc_fence_after();
@@ -116,11 +123,12 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
                 for (int kk = 0; kk < RTC_BK / 16; ++kk)
                     umma_bf16_ss(tmem_base, umma_desc_sw128(sa + kk * 32),
                                  umma_desc_sw128(sb + kk * 32), idesc,
-                                 (kb > kb0 || kk > 0) ? 1u : 0u);
+                                 (i > 0 || kk > 0) ? 1u : 0u);
                 umma_commit(&empty[s]);
             }
             umma_commit(tfull); // arrives once every MMA issued above has completed
         }
+        __syncwarp();
     } else if (warp >= 4) {
         // Drain the accumulator: TMEM lane = token row, column = expert.
         const int q = warp & 3;
