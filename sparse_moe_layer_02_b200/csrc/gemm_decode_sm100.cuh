@@ -344,16 +344,19 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
                             float sum[8];
 #pragma unroll
                             for (int h = 0; h < 8; ++h) sum[h] = 0.f;
-                            for (int j = 0; j < a.k; ++j) {
-                                const int p = a.pos_of[(size_t)n * a.k + j];
-                                if (p < 0) continue;
-                                const uint4 w4 = __ldcg(reinterpret_cast<const uint4 *>(
-                                    a.slot + (size_t)p * a.ld_r + col));
-                                float lo, hi;
-                                unpack_bf16x2(w4.x, lo, hi); sum[0] += lo; sum[1] += hi;
-                                unpack_bf16x2(w4.y, lo, hi); sum[2] += lo; sum[3] += hi;
-                                unpack_bf16x2(w4.z, lo, hi); sum[4] += lo; sum[5] += hi;
-                                unpack_bf16x2(w4.w, lo, hi); sum[6] += lo; sum[7] += hi;
+                            // eight slots fetched before any is added; adds in slot order
+                            for (int jb = 0; jb < a.k; jb += 8) {
+                                uint4 w[8];
+#pragma unroll
+                                for (int jj = 0; jj < 8; ++jj) {
+                                    const int j = jb + jj;
+                                    const int p = j < a.k ? a.pos_of[(size_t)n * a.k + j] : -1;
+                                    w[jj] = p >= 0 ? __ldcg(reinterpret_cast<const uint4 *>(
+                                                         a.slot + (size_t)p * a.ld_r + col))
+                                                   : make_uint4(0u, 0u, 0u, 0u);
+                                }
+#pragma unroll
+                                for (int jj = 0; jj < 8; ++jj) acc_bf16x8(sum, w[jj]);
                             }
                             const float *o = epi + tk * DEC_EPI_LD + pc * 8;
                             uint32_t pk[4];

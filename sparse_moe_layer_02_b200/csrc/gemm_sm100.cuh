@@ -125,8 +125,19 @@ __device__ __forceinline__ void store_row_chunk_bf16(__nv_bfloat16 *row_ptr, int
         if (col + 8 * q < ncols) dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
 }
 
+// Adds the eight bf16 values of w into acc (fp32).
+__device__ __forceinline__ void acc_bf16x8(float (&acc)[8], const uint4 &w) {
+    float lo, hi;
+    unpack_bf16x2(w.x, lo, hi); acc[0] += lo; acc[1] += hi;
+    unpack_bf16x2(w.y, lo, hi); acc[2] += lo; acc[3] += hi;
+    unpack_bf16x2(w.z, lo, hi); acc[4] += lo; acc[5] += hi;
+    unpack_bf16x2(w.w, lo, hi); acc[6] += lo; acc[7] += hi;
+}
+
 // y[n] = sum_{j<k} slot[pos(n, j)] (slot order) + osh[n], one warp per row, each
-// lane two 8-column pieces at a time so 2(k+2) 16-byte loads are in flight.
+// lane two 8-column pieces at a time.  The slot rows are fetched eight slots at
+// a time before any of them is added, so 16 slot loads and the shared row are in
+// flight per lane; the adds then run in slot order (a missing slot adds +0).
 __device__ __forceinline__ void combine_rows(const GemmArgs &a, int gwarp, int nwarps, int lane) {
     const int pieces = a.ncols_s / 8;
     for (int n = gwarp; n < a.N; n += nwarps) {
@@ -134,34 +145,46 @@ __device__ __forceinline__ void combine_rows(const GemmArgs &a, int gwarp, int n
         // Uniform trip count across the warp: the shuffles below need every lane.
         for (int pbase = 0; pbase < pieces; pbase += 64) {
             const int p0 = pbase + lane;
+            float4 o[2][2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int pc = p0 + 32 * u;
+                if (pc < pieces) {
+                    const float4 *op = reinterpret_cast<const float4 *>(a.osh + (size_t)n * a.ld_s + pc * 8);
+                    o[u][0] = __ldcg(op);
+                    o[u][1] = __ldcg(op + 1);
+                }
+            }
             float sum[2][8];
 #pragma unroll
             for (int u = 0; u < 2; ++u)
 #pragma unroll
                 for (int h = 0; h < 8; ++h) sum[u][h] = 0.f;
-            for (int j = 0; j < a.k; ++j) {
-                const int p = __shfl_sync(0xffffffffu, my_pos, j);
-                if (p < 0) continue;
-                const __nv_bfloat16 *srow = a.slot + (size_t)p * a.ld_r;
+            for (int jb = 0; jb < a.k; jb += 8) {
+                uint4 w[8][2];
 #pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const int pc = p0 + 32 * u;
-                    if (pc < pieces) {
-                        const uint4 w4 = __ldcg(reinterpret_cast<const uint4 *>(srow + pc * 8));
-                        float lo, hi;
-                        unpack_bf16x2(w4.x, lo, hi); sum[u][0] += lo; sum[u][1] += hi;
-                        unpack_bf16x2(w4.y, lo, hi); sum[u][2] += lo; sum[u][3] += hi;
-                        unpack_bf16x2(w4.z, lo, hi); sum[u][4] += lo; sum[u][5] += hi;
-                        unpack_bf16x2(w4.w, lo, hi); sum[u][6] += lo; sum[u][7] += hi;
+                for (int jj = 0; jj < 8; ++jj) {
+                    const int j = jb + jj;
+                    const int p = __shfl_sync(0xffffffffu, my_pos, j & 31);
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const int pc = p0 + 32 * u;
+                        w[jj][u] = make_uint4(0u, 0u, 0u, 0u);
+                        if (j < a.k && p >= 0 && pc < pieces)
+                            w[jj][u] = __ldcg(reinterpret_cast<const uint4 *>(
+                                a.slot + (size_t)p * a.ld_r + pc * 8));
                     }
                 }
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj)
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) acc_bf16x8(sum[u], w[jj][u]);
             }
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
                 const int pc = p0 + 32 * u;
                 if (pc < pieces) {
-                    const float4 *o = reinterpret_cast<const float4 *>(a.osh + (size_t)n * a.ld_s + pc * 8);
-                    const float4 o0 = __ldcg(o), o1 = __ldcg(o + 1);
+                    const float4 o0 = o[u][0], o1 = o[u][1];
                     const uint4 out = make_uint4(pack_bf16x2(sum[u][0] + o0.x, sum[u][1] + o0.y),
                                                  pack_bf16x2(sum[u][2] + o0.z, sum[u][3] + o0.w),
                                                  pack_bf16x2(sum[u][4] + o1.x, sum[u][5] + o1.y),

@@ -6,7 +6,7 @@
 #include <atomic>
 #include <mutex>
 
-#include "../../include/moe.h"
+#include "moe.h"
 #include "common.cuh"
 #include "dispatch.cuh"
 #include "gemm_decode_sm100.cuh"

@@ -26,7 +26,7 @@
 
 #include <mutex>
 
-#include "../../include/moe.h"
+#include "moe.h"
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[MOE_NOALLOC_SCRATCH_BYTES];
 
