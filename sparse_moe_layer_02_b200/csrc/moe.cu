@@ -213,20 +213,21 @@ int launch_router_x(const RouterParams &p, cudaStream_t st) {
     return launch_router_t<XT, WT, 16>(p, st);
 }
 
-template <int EV>
+template <int EV, bool WF32>
 int launch_router_tc_t(const CUtensorMap &mX, const CUtensorMap &mW, const RouterParams &p, int clk,
                        cudaStream_t st) {
+    constexpr int smem = RtcCfg<WF32>::SMEM;
     static bool attr_set = false;
     if (!attr_set) {
-        if (cudaFuncSetAttribute(router_tc_kernel<EV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 RTC_SMEM_BYTES) != cudaSuccess)
+        if (cudaFuncSetAttribute(router_tc_kernel<EV, WF32>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
             return MOE_ERR_CUDA;
         attr_set = true;
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(clk, (p.N + RTC_BM - 1) / RTC_BM, 1);
     cfg.blockDim = dim3(RTC_THREADS, 1, 1);
-    cfg.dynamicSmemBytes = RTC_SMEM_BYTES;
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -235,25 +236,32 @@ int launch_router_tc_t(const CUtensorMap &mX, const CUtensorMap &mW, const Route
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, router_tc_kernel<EV>, mX, mW, p, g_wait_limit_ns) != cudaSuccess)
+    if (cudaLaunchKernelEx(&cfg, router_tc_kernel<EV, WF32>, mX, mW, p, g_wait_limit_ns) !=
+        cudaSuccess)
         return MOE_ERR_CUDA;
     return launch_status();
 }
 
-// Tensor-core router for bf16 x and bf16 W_g with 16 <= E <= 256, E % 16 == 0.
+// Tensor-core router for bf16 x with a bf16 W_g (16 <= E <= 256) or an fp32 W_g
+// (16 <= E <= 192, three-way bf16 split); E % 16 == 0.
+template <bool WF32>
 int launch_router_tc(const RouterParams &p, int sms, cudaStream_t st) {
     CUtensorMap mX, mW;
-    if (!make_map(&mX, p.x, p.D, p.N, p.D, RTC_BM) || !make_map(&mW, p.W_g, p.D, p.E, p.D, p.E))
+    if (!make_map(&mX, p.x, p.D, p.N, p.D, RTC_BM)) return MOE_ERR_CUDA;
+    if (WF32) {
+        mW = mX; // unused: the fp32 matrix is read and split by the kernel's own warps
+    } else if (!make_map(&mW, p.W_g, p.D, p.E, p.D, p.E)) {
         return MOE_ERR_CUDA;
+    }
     const int tblocks = (p.N + RTC_BM - 1) / RTC_BM;
     // K-split cluster size: a power of two (so it divides the 128 tokens of a
     // block) chosen to put about one CTA on every SM, at most 8.
     int clk = 1;
     while (clk < 8 && 2 * clk * tblocks <= sms) clk *= 2;
-    if (p.E <= 32) return launch_router_tc_t<1>(mX, mW, p, clk, st);
-    if (p.E <= 64) return launch_router_tc_t<2>(mX, mW, p, clk, st);
-    if (p.E <= 128) return launch_router_tc_t<4>(mX, mW, p, clk, st);
-    return launch_router_tc_t<8>(mX, mW, p, clk, st);
+    if (p.E <= 32) return launch_router_tc_t<1, WF32>(mX, mW, p, clk, st);
+    if (p.E <= 64) return launch_router_tc_t<2, WF32>(mX, mW, p, clk, st);
+    if (p.E <= 128) return launch_router_tc_t<4, WF32>(mX, mW, p, clk, st);
+    return launch_router_tc_t<8, WF32>(mX, mW, p, clk, st);
 }
 
 template <int KIND>
@@ -397,9 +405,10 @@ int moe_router(const void *x, int x_dtype, const void *W_g, int wg_dtype, const 
     p.topk_idx = topk_idx;
     p.topk_w = topk_w;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (x_dtype == MOE_BF16 && wg_dtype == MOE_BF16 && E % 16 == 0 && E >= 16 && E <= 256 &&
-        D % 8 == 0)
-        return launch_router_tc(p, dev->sms, st);
+    if (x_dtype == MOE_BF16 && E % 16 == 0 && E >= 16 && D % 8 == 0) {
+        if (wg_dtype == MOE_BF16 && E <= 256) return launch_router_tc<false>(p, dev->sms, st);
+        if (wg_dtype == MOE_F32 && E <= RTC_MAXE_F32) return launch_router_tc<true>(p, dev->sms, st);
+    }
     if (x_dtype == MOE_F32 && wg_dtype == MOE_F32) return launch_router_x<float, float>(p, st);
     if (x_dtype == MOE_BF16 && wg_dtype == MOE_F32) return launch_router_x<__nv_bfloat16, float>(p, st);
     if (x_dtype == MOE_BF16 && wg_dtype == MOE_BF16)

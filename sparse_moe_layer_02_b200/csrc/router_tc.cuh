@@ -1,15 +1,22 @@
-// Router logits on the tensor cores for bf16 tokens and a bf16 router matrix
-// ("GLM-4.5 Group Router", How it works: r = x W_g^T in float32; bf16 x bf16
-// products are exact in fp32 and tcgen05 accumulates in fp32).
+// Router logits on the tensor cores ("GLM-4.5 Group Router", How it works:
+// r = x W_g^T in float32) for bf16 tokens and a bf16 or fp32 router matrix.
+//
+// bf16 W_g: bf16 x bf16 products are exact in fp32 and tcgen05 accumulates in
+// fp32.  fp32 W_g: every element is split into three bf16 parts,
+// w = w1 + w2 + w3 with w1 = bf16(w), w2 = bf16(w - w1), w3 = bf16(w - w1 - w2)
+// (each residual is exact in fp32, and the split reproduces w to 2^-27 relative,
+// finer than fp32 rounding), and x W_g^T is accumulated as three bf16 products
+// into the same fp32 accumulator.  Idle warps do the split into shared memory
+// while the TMA fetches the tokens.
 //
 // One cluster of CLK CTAs per 128 tokens: CTA r multiplies the tokens' rows by
 // W_g over the r-th slice of the hidden dimension (M = 128 tokens, N = E
-// experts, K = 16 per instruction; TMA-fed 4-stage ring; one 128 x E fp32
-// accumulator in TMEM).  The partial logits go to shared memory; after a cluster
-// barrier, warps take whole tokens, sum the CLK partial rows in rank order
-// (distributed shared memory; a fixed order, so the result is deterministic) and
-// run the same warp-shuffle selection as the CUDA-core router.  CLK = 1 for
-// large batches; small batches split K over up to 8 CTAs so more SMs stream W_g.
+// experts, K = 16 per instruction; one 128 x E fp32 accumulator in TMEM).  The
+// partial logits go to shared memory; after a cluster barrier, warps take whole
+// tokens, sum the CLK partial rows in rank order (distributed shared memory; a
+// fixed order, so the result is deterministic) and run the same warp-shuffle
+// selection as the CUDA-core router.  CLK = 1 for large batches; small batches
+// split K over up to 8 CTAs so more SMs stream W_g.
 #pragma once
 
 #include <cooperative_groups.h>
@@ -21,31 +28,72 @@ namespace moe {
 
 constexpr int RTC_BM = 128;
 constexpr int RTC_BK = 64;
-constexpr int RTC_STAGES = 4;
-constexpr int RTC_THREADS = 256;   // warp 0 TMA, warp 1 MMA, warps 4-7 TMEM drain, all select
-constexpr int RTC_A_BYTES = RTC_BM * RTC_BK * 2;     // 16 KiB
-constexpr int RTC_B_BYTES_MAX = 256 * RTC_BK * 2;    // 32 KiB (E <= 256)
-constexpr int RTC_STAGE_BYTES = RTC_A_BYTES + RTC_B_BYTES_MAX;
-constexpr int RTC_PART_LD = 257;                     // floats per token row of the partials
-constexpr int RTC_SMEM_BYTES = 1024 + RTC_STAGES * RTC_STAGE_BYTES + 256 +
-                               (RTC_THREADS / 32) * ROUTER_MAXV * 32 * 4;
-static_assert(RTC_BM * RTC_PART_LD * 4 <= RTC_STAGES * RTC_STAGE_BYTES,
-              "partial logits reuse the operand ring");
+constexpr int RTC_THREADS = 256;  // warp 0 TMA, warp 1 MMA, warps 2-7 split (fp32), 4-7 drain
+constexpr int RTC_A_BYTES = RTC_BM * RTC_BK * 2;  // 16 KiB
+constexpr int RTC_PART_LD = 257;                  // floats per token row of the partials
+constexpr int RTC_MAXE_F32 = 192;                 // largest E of the fp32-W_g variant
 
-template <int EV>
+template <bool WF32> struct RtcCfg {
+    static constexpr int STAGES = WF32 ? 2 : 4;
+    static constexpr int B_PART = (WF32 ? RTC_MAXE_F32 : 256) * RTC_BK * 2; // one bf16 B tile
+    static constexpr int B_BYTES = (WF32 ? 3 : 1) * B_PART;
+    static constexpr int STAGE_BYTES = RTC_A_BYTES + B_BYTES;
+    static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + 256 +
+                                (RTC_THREADS / 32) * ROUTER_MAXV * 32 * 4;
+    static_assert(STAGE_BYTES % 1024 == 0, "stages stay 1024-byte aligned");
+    static_assert(RTC_BM * RTC_PART_LD * 4 <= STAGES * STAGE_BYTES,
+                  "partial logits reuse the operand ring");
+};
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Split 8 fp32 router weights into three bf16 parts, written as one 16-byte chunk
+// of each part's K-major tile with the 128-byte swizzle the MMA descriptor uses.
+__device__ __forceinline__ void split_store(uint8_t *b0, int row, int chunk, const float4 &u,
+                                            const float4 &v, int part_bytes) {
+    const float w[8] = {u.x, u.y, u.z, u.w, v.x, v.y, v.z, v.w};
+    uint32_t p1[4], p2[4], p3[4];
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+        float a1[2], a2[2], a3[2];
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            const float x0 = w[2 * h + q];
+            const __nv_bfloat16 h1 = __float2bfloat16_rn(x0);
+            const float r1 = x0 - __bfloat162float(h1);
+            const __nv_bfloat16 h2 = __float2bfloat16_rn(r1);
+            const float r2 = r1 - __bfloat162float(h2);
+            a1[q] = __bfloat162float(h1);
+            a2[q] = __bfloat162float(h2);
+            a3[q] = r2;
+        }
+        p1[h] = pack_bf16x2(a1[0], a1[1]);
+        p2[h] = pack_bf16x2(a2[0], a2[1]);
+        p3[h] = pack_bf16x2(a3[0], a3[1]);
+    }
+    const int off = row * 128 + ((chunk ^ (row & 7)) << 4);
+    *reinterpret_cast<uint4 *>(b0 + off) = make_uint4(p1[0], p1[1], p1[2], p1[3]);
+    *reinterpret_cast<uint4 *>(b0 + part_bytes + off) = make_uint4(p2[0], p2[1], p2[2], p2[3]);
+    *reinterpret_cast<uint4 *>(b0 + 2 * part_bytes + off) = make_uint4(p3[0], p3[1], p3[2], p3[3]);
+}
+
+template <int EV, bool WF32>
 __global__ void __launch_bounds__(RTC_THREADS, 1)
     router_tc_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mW,
                      const RouterParams p, uint64_t limit) {
+    using C = RtcCfg<WF32>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint8_t *ring = smem;
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + RTC_STAGES * RTC_STAGE_BYTES);
-    uint64_t *empty = full + RTC_STAGES;
-    uint64_t *tfull = empty + RTC_STAGES;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::STAGES * C::STAGE_BYTES);
+    uint64_t *empty = full + C::STAGES;
+    uint64_t *tfull = empty + C::STAGES;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tfull + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    float *spbuf = reinterpret_cast<float *>(smem + RTC_STAGES * RTC_STAGE_BYTES + 256);
+    float *spbuf = reinterpret_cast<float *>(smem + C::STAGES * C::STAGE_BYTES + 256);
     float *part = reinterpret_cast<float *>(ring); // [128][RTC_PART_LD] after the main loop
 
     cg::cluster_group cluster = cg::this_cluster();
@@ -57,17 +105,17 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
     const int KB = (p.D + RTC_BK - 1) / RTC_BK;
     const int kper = (KB + CLK - 1) / CLK;
     const int kb0 = rank * kper, kb1 = min(KB, kb0 + kper);
-    const uint32_t b_bytes = (uint32_t)E * RTC_BK * 2;
-    // Every CTA reads the same W_g slices; rotating the k-block order by the token
-    // block spreads concurrent reads over different L2 lines instead of having all
-    // CTAs request the same 32 KiB at once.
-    const int nkb = kb1 - kb0;
-    const int rot = nkb > 0 ? (int)(blockIdx.y % (unsigned)nkb) : 0;
     const uint32_t tmem_cols = E <= 32 ? 32 : E <= 64 ? 64 : E <= 128 ? 128 : 256;
+    // Every CTA reads the same W_g slices; rotating the k-block order by the token
+    // block spreads concurrent reads over different L2 lines.
+    const int nkb = kb1 > kb0 ? kb1 - kb0 : 0;
+    const int rot = nkb > 0 ? (int)(blockIdx.y % (unsigned)nkb) : 0;
+    auto kb_of = [&](int i) { return kb0 + (i + rot < nkb ? i + rot : i + rot - nkb); };
+    constexpr int NCONV = 6; // warps 2-7 split fp32 W_g
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < RTC_STAGES; ++s) {
-            mbar_init(&full[s], 1);
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(&full[s], WF32 ? 1 + NCONV : 1);
             mbar_init(&empty[s], 1);
         }
         mbar_init(tfull, 1);
@@ -76,7 +124,7 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
     }
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&mX);
-        tma_prefetch_desc(&mW);
+        if (!WF32) tma_prefetch_desc(&mW);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, tmem_cols);
@@ -92,19 +140,19 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
             uint32_t it = 0;
             bool ok = true;
             for (int i = 0; i < nkb; ++i, ++it) {
-                const int kb = kb0 + (i + rot < nkb ? i + rot : i + rot - nkb);
-                const uint32_t s = it % RTC_STAGES, ph = (it / RTC_STAGES) & 1;
+                const int kb = kb_of(i);
+                const uint32_t s = it % C::STAGES, ph = (it / C::STAGES) & 1;
                 if (!mbar_wait(&empty[s], ph ^ 1, limit, abort_flag, 300)) { ok = false; break; }
-                uint8_t *sa = ring + s * RTC_STAGE_BYTES;
-                mbar_arrive_expect_tx(&full[s], RTC_A_BYTES + b_bytes);
+                uint8_t *sa = ring + s * C::STAGE_BYTES;
+                mbar_arrive_expect_tx(&full[s], RTC_A_BYTES + (WF32 ? 0u : (uint32_t)E * RTC_BK * 2));
                 tma_load_2d(&mX, &full[s], sa, kb * RTC_BK, t0);
-                tma_load_2d(&mW, &full[s], sa + RTC_A_BYTES, kb * RTC_BK, 0);
+                if (!WF32) tma_load_2d(&mW, &full[s], sa + RTC_A_BYTES, kb * RTC_BK, 0);
             }
             if (!ok) {
-                const uint32_t first = it > RTC_STAGES ? it - RTC_STAGES : 0;
+                const uint32_t first = it > (uint32_t)C::STAGES ? it - C::STAGES : 0;
                 for (uint32_t j = first; j < it; ++j) {
                     volatile int no_abort = 0;
-                    mbar_wait(&full[j % RTC_STAGES], (j / RTC_STAGES) & 1, 10000000ull, &no_abort, 301);
+                    mbar_wait(&full[j % C::STAGES], (j / C::STAGES) & 1, 10000000ull, &no_abort, 301);
                 }
             }
         }
@@ -114,22 +162,62 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
             const uint32_t idesc = umma_idesc_bf16(RTC_BM, E);
             uint32_t it = 0;
             for (int i = 0; i < nkb; ++i, ++it) {
-                const uint32_t s = it % RTC_STAGES, ph = (it / RTC_STAGES) & 1;
+                const uint32_t s = it % C::STAGES, ph = (it / C::STAGES) & 1;
                 if (!mbar_wait(&full[s], ph, limit, abort_flag, 310)) break;
                 tc_fence_after();
-                const uint32_t sa = smem_u32(ring + s * RTC_STAGE_BYTES);
+                const uint32_t sa = smem_u32(ring + s * C::STAGE_BYTES);
                 const uint32_t sb = sa + RTC_A_BYTES;
 #pragma unroll
-                for (int kk = 0; kk < RTC_BK / 16; ++kk)
-                    umma_bf16_ss(tmem_base, umma_desc_sw128(sa + kk * 32),
-                                 umma_desc_sw128(sb + kk * 32), idesc,
-                                 (i > 0 || kk > 0) ? 1u : 0u);
+                for (int kk = 0; kk < RTC_BK / 16; ++kk) {
+#pragma unroll
+                    for (int part_i = 0; part_i < (WF32 ? 3 : 1); ++part_i)
+                        umma_bf16_ss(tmem_base, umma_desc_sw128(sa + kk * 32),
+                                     umma_desc_sw128(sb + part_i * C::B_PART + kk * 32), idesc,
+                                     (i > 0 || kk > 0 || part_i > 0) ? 1u : 0u);
+                }
                 umma_commit(&empty[s]);
             }
             umma_commit(tfull); // arrives once every MMA issued above has completed
         }
         __syncwarp();
-    } else if (warp >= 4) {
+    } else if (WF32) {
+        // Split fp32 W_g into three bf16 tiles per stage (warps 2-7).
+        const int cw = warp - 2, ct = cw * 32 + lane;
+        const float *W = static_cast<const float *>(p.W_g);
+        uint32_t it = 0;
+        for (int i = 0; i < nkb; ++i, ++it) {
+            const int kb = kb_of(i);
+            const uint32_t s = it % C::STAGES, ph = (it / C::STAGES) & 1;
+            bool ok = true;
+            if (lane == 0) ok = mbar_wait(&empty[s], ph ^ 1, limit, abort_flag, 330);
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (!ok) break;
+            uint8_t *b0 = ring + s * C::STAGE_BYTES + RTC_A_BYTES;
+            const int k0 = kb * RTC_BK;
+            for (int item = ct; item < E * 8; item += NCONV * 32) {
+                const int row = item >> 3, chunk = item & 7;
+                const int kk = k0 + chunk * 8;
+                float4 u = make_float4(0.f, 0.f, 0.f, 0.f), v = u;
+                const float *src = W + (size_t)row * p.D + kk;
+                if (kk + 8 <= p.D) {
+                    u = __ldg(reinterpret_cast<const float4 *>(src));
+                    v = __ldg(reinterpret_cast<const float4 *>(src) + 1);
+                } else {
+                    float t[8];
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) t[q] = kk + q < p.D ? src[q] : 0.f;
+                    u = make_float4(t[0], t[1], t[2], t[3]);
+                    v = make_float4(t[4], t[5], t[6], t[7]);
+                }
+                split_store(b0, row, chunk, u, v, C::B_PART);
+            }
+            fence_proxy_async_smem(); // generic-proxy stores -> visible to the tensor core
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&full[s]);
+        }
+        __syncwarp();
+    }
+    if (warp >= 4) {
         // Drain the accumulator: TMEM lane = token row, column = expert.
         const int q = warp & 3;
         const int row = q * 32 + lane;
@@ -138,7 +226,7 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
         have = __shfl_sync(0xffffffffu, have ? 1 : 0, 0) != 0;
         __syncwarp();
         if (have) tc_fence_after();
-        const bool empty_k = kb0 >= kb1;
+        const bool empty_k = nkb == 0;
         for (int c0 = 0; c0 < E; c0 += 32) {
             uint32_t v[32];
             if (have) {

@@ -100,6 +100,19 @@ def test_router_shapes(E, G, tg, k):
     assert rep["unexplained"] == 0 and rep["max_w_err_over_alpha"] <= W_TOL
 
 
+@pytest.mark.parametrize("E,G,tg,k,D", [(64, 8, 3, 6, 264), (192, 1, 1, 8, 328), (160, 1, 1, 8, 264),
+                                        (208, 1, 1, 8, 264), (48, 4, 2, 4, 4096)])
+def test_router_fp32_matrix_shapes(E, G, tg, k, D):
+    # bf16 tokens with an fp32 router matrix: the tensor-core path splits W_g into
+    # three bf16 parts (E <= 192), larger E use the CUDA-core path.
+    cfg = CONFIGS["glm45_prefill"].with_(N=333, D=D, E=E, n_group=G, topk_group=tg, k=k)
+    x, wg, b, _ = router_inputs(cfg, seed=E + D, device=DEV)
+    idx, w = moe.moe_router(x, wg, b, G, tg, k, True, cfg.alpha)
+    orc = oracle.router(x.cpu(), wg.cpu(), b.cpu(), G, tg, k, True, cfg.alpha)
+    rep = compare_routing(idx, w, orc, b, cfg.alpha)
+    assert rep["unexplained"] == 0 and rep["max_w_err_over_alpha"] <= W_TOL
+
+
 # ----------------------------------------------------------------------------- forward
 SMALL = {
     # name: (base config, overrides)
