@@ -278,6 +278,8 @@ def main():
     w = torch.empty((N, cfg.k), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
     kernels = BF16_KERNELS if cfg.dtype == torch.bfloat16 else F32_KERNELS
+    if cfg.N * cfg.k <= 2048:  # one fused dispatch kernel; its marks fill the first slot
+        kernels = ["dispatch", "_", "_"] + kernels[3:]
 
     def step(x):
         moe.moe_router(x, inp.W_g, inp.b, cfg.n_group, cfg.topk_group, cfg.k, cfg.norm_topk_prob,
@@ -341,7 +343,8 @@ def main():
     # Per-kernel durations over the timed region.
     per = {"router": sum(evs[s][0].elapsed_time(evs[s][1]) for s in range(K)) / K}
     for i, name in enumerate(kernels):
-        per[name] = sum(evs[s][1 + i].elapsed_time(evs[s][2 + i]) for s in range(K)) / K
+        if name != "_":
+            per[name] = sum(evs[s][1 + i].elapsed_time(evs[s][2 + i]) for s in range(K)) / K
     dom = max(per, key=per.get)
     peaks, peak_src = load_peaks()
     flops, byts = kernel_work(cfg, dom, hit)

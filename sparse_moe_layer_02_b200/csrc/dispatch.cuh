@@ -154,6 +154,110 @@ __global__ void __launch_bounds__(DISPATCH_THREADS) dispatch_scatter_kernel(cons
     }
 }
 
+// Whole dispatch (count, scan, scatter) in one CTA for batches of at most
+// DISPATCH_SMALL_IDS ids, as at decode: same results as the three kernels above
+// (stable positions ordered by expert, then token, then slot).
+constexpr int DISPATCH_SMALL_IDS = 2048;
+constexpr int DISPATCH_SMALL_THREADS = 512;
+
+__global__ void __launch_bounds__(DISPATCH_SMALL_THREADS) dispatch_small_kernel(const DispatchParams p) {
+    constexpr int NW = DISPATCH_SMALL_THREADS / 32;
+    __shared__ int hist[DISPATCH_MAXE];
+    __shared__ int cursor[DISPATCH_MAXE];
+    __shared__ int wcnt[NW][DISPATCH_MAXE];
+    __shared__ int wsum[NW];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int total = p.N * p.k;
+    for (int e = tid; e < p.E; e += DISPATCH_SMALL_THREADS) {
+        hist[e] = 0;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) wcnt[w][e] = 0;
+    }
+    __syncthreads();
+    for (int i = tid; i < total; i += DISPATCH_SMALL_THREADS) {
+        const int e = p.topk_idx[i];
+        if (e >= 0 && e < p.E)
+            atomicAdd(&hist[e], 1);
+        else if (e != p.E)
+            record_error(DEV_BAD_INDEX, 11);
+    }
+    __syncthreads();
+    // exclusive scan of tiles per expert (thread e owns expert e; E <= 512)
+    const int e = tid;
+    const int cnt = e < p.E ? hist[e] : 0;
+    const int tiles = (cnt + p.tile_rows - 1) / p.tile_rows;
+    int v = tiles;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, v, off);
+        if (lane >= off) v += n;
+    }
+    if (lane == 31) wsum[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+        int w = lane < NW ? wsum[lane] : 0;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int n = __shfl_up_sync(0xffffffffu, w, off);
+            if (lane >= off) w += n;
+        }
+        if (lane < NW) wsum[lane] = w;
+    }
+    __syncthreads();
+    const int incl = v + (warp > 0 ? wsum[warp - 1] : 0);
+    const int excl = incl - tiles;
+    if (e < p.E) {
+        p.counts[e] = cnt;
+        p.tile_off[e] = excl;
+        cursor[e] = excl * p.tile_rows;
+    }
+    if (e == p.E - 1) {
+        p.tile_off[p.E] = incl;
+        p.meta[0] = 0;
+        p.meta[1] = incl * p.tile_rows;
+        p.meta[2] = incl;
+    }
+    __syncthreads();
+    // stable positions, DISPATCH_SMALL_THREADS ids per round
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    for (int base = 0; base < total; base += DISPATCH_SMALL_THREADS) {
+        const int i = base + tid;
+        const bool valid = i < total;
+        int key = -1;
+        if (valid) {
+            const int ee = p.topk_idx[i];
+            key = (ee >= 0 && ee < p.E) ? ee : -1;
+        }
+        const uint32_t peers = __match_any_sync(0xffffffffu, key);
+        const int rank = __popc(peers & lt_mask);
+        if (key >= 0 && rank == 0) wcnt[warp][key] = __popc(peers);
+        __syncthreads();
+        int pos = -1;
+        if (key >= 0) {
+            pos = cursor[key] + rank;
+            for (int w = 0; w < warp; ++w) pos += wcnt[w][key];
+        }
+        __syncthreads();
+        for (int ee = tid; ee < p.E; ee += DISPATCH_SMALL_THREADS) {
+            int add = 0;
+#pragma unroll
+            for (int w = 0; w < NW; ++w) {
+                add += wcnt[w][ee];
+                wcnt[w][ee] = 0;
+            }
+            cursor[ee] += add;
+        }
+        if (valid) {
+            p.pos_of[i] = pos;
+            if (pos >= 0) {
+                p.perm_tok[pos] = i / p.k;
+                p.w_perm[pos] = p.topk_w[i];
+            }
+        }
+        __syncthreads();
+    }
+}
+
 // Padding rows (beyond an expert's count inside its last tile) carry no
 // token; perm_tok / w_perm are left unset there and every reader checks this.
 __device__ __forceinline__ int expert_of_tile(const int *tile_off, int E, int mt) {

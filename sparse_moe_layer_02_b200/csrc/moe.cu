@@ -217,13 +217,34 @@ template <int EV, bool WF32>
 int launch_router_tc_t(const CUtensorMap &mX, const CUtensorMap &mW, const RouterParams &p, int clk,
                        cudaStream_t st) {
     constexpr int smem = RtcCfg<WF32>::SMEM;
-    static bool attr_set = false;
-    if (!attr_set) {
+    static int max_clk = 0; // largest cluster size this kernel can be launched with
+    if (!max_clk) {
         if (cudaFuncSetAttribute(router_tc_kernel<EV, WF32>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
             return MOE_ERR_CUDA;
-        attr_set = true;
+        max_clk = 8;
+        if (cudaFuncSetAttribute(router_tc_kernel<EV, WF32>,
+                                 cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
+            cudaLaunchConfig_t q = {};
+            q.gridDim = dim3(RTC_MAX_CLK, 1, 1);
+            q.blockDim = dim3(RTC_THREADS, 1, 1);
+            q.dynamicSmemBytes = smem;
+            cudaLaunchAttribute qa[1];
+            qa[0].id = cudaLaunchAttributeClusterDimension;
+            qa[0].val.clusterDim.x = RTC_MAX_CLK;
+            qa[0].val.clusterDim.y = 1;
+            qa[0].val.clusterDim.z = 1;
+            q.attrs = qa;
+            q.numAttrs = 1;
+            int clusters = 0;
+            if (cudaOccupancyMaxActiveClusters(&clusters, router_tc_kernel<EV, WF32>, &q) ==
+                    cudaSuccess &&
+                clusters > 0)
+                max_clk = RTC_MAX_CLK;
+        }
+        cudaGetLastError(); // a refused query is not an error of this call
     }
+    if (clk > max_clk) clk = max_clk;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(clk, (p.N + RTC_BM - 1) / RTC_BM, 1);
     cfg.blockDim = dim3(RTC_THREADS, 1, 1);
@@ -255,9 +276,10 @@ int launch_router_tc(const RouterParams &p, int sms, cudaStream_t st) {
     }
     const int tblocks = (p.N + RTC_BM - 1) / RTC_BM;
     // K-split cluster size: a power of two (so it divides the 128 tokens of a
-    // block) chosen to put about one CTA on every SM, at most 8.
+    // block) chosen to put about one CTA on every SM, at most 16 (8 where the
+    // device cannot co-schedule 16-CTA clusters of this kernel).
     int clk = 1;
-    while (clk < 8 && 2 * clk * tblocks <= sms) clk *= 2;
+    while (clk < RTC_MAX_CLK && 2 * clk * tblocks <= sms) clk *= 2;
     if (p.E <= 32) return launch_router_tc_t<1, WF32>(mX, mW, p, clk, st);
     if (p.E <= 64) return launch_router_tc_t<2, WF32>(mX, mW, p, clk, st);
     if (p.E <= 128) return launch_router_tc_t<4, WF32>(mX, mW, p, clk, st);
@@ -465,12 +487,20 @@ int moe_forward(const void *x, const void *gate_up, const void *down, const void
     dp.perm_tok = reinterpret_cast<int32_t *>(ws + L.perm_tok);
     dp.w_perm = reinterpret_cast<float *>(ws + L.w_perm);
 
-    dispatch_count_kernel<<<L.nchunks, DISPATCH_THREADS, 0, st>>>(dp);
-    if ((rc = launched(prof)) != MOE_OK) return rc;
-    dispatch_scan_kernel<<<1, DISPATCH_MAXE, 0, st>>>(dp);
-    if ((rc = launched(prof)) != MOE_OK) return rc;
-    dispatch_scatter_kernel<<<L.nchunks, DISPATCH_THREADS, 0, st>>>(dp);
-    if ((rc = launched(prof)) != MOE_OK) return rc;
+    if ((size_t)N * k <= DISPATCH_SMALL_IDS) {
+        // one CTA does count, scan and scatter (the three profiling marks coincide)
+        dispatch_small_kernel<<<1, DISPATCH_SMALL_THREADS, 0, st>>>(dp);
+        if ((rc = launched(prof)) != MOE_OK) return rc;
+        prof.mark();
+        prof.mark();
+    } else {
+        dispatch_count_kernel<<<L.nchunks, DISPATCH_THREADS, 0, st>>>(dp);
+        if ((rc = launched(prof)) != MOE_OK) return rc;
+        dispatch_scan_kernel<<<1, DISPATCH_MAXE, 0, st>>>(dp);
+        if ((rc = launched(prof)) != MOE_OK) return rc;
+        dispatch_scatter_kernel<<<L.nchunks, DISPATCH_THREADS, 0, st>>>(dp);
+        if ((rc = launched(prof)) != MOE_OK) return rc;
+    }
 
     if (dtype == MOE_F32) {
         SimtArgs a;

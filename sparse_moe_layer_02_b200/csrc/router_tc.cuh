@@ -16,7 +16,7 @@
 // tokens, sum the CLK partial rows in rank order (distributed shared memory; a
 // fixed order, so the result is deterministic) and run the same warp-shuffle
 // selection as the CUDA-core router.  CLK = 1 for large batches; small batches
-// split K over up to 8 CTAs so more SMs stream W_g.
+// split K over up to 16 CTAs so more SMs stream W_g.
 #pragma once
 
 #include <cooperative_groups.h>
@@ -32,6 +32,7 @@ constexpr int RTC_THREADS = 256;  // warp 0 TMA, warp 1 MMA, warps 2-7 split (fp
 constexpr int RTC_A_BYTES = RTC_BM * RTC_BK * 2;  // 16 KiB
 constexpr int RTC_PART_LD = 257;                  // floats per token row of the partials
 constexpr int RTC_MAXE_F32 = 192;                 // largest E of the fp32-W_g variant
+constexpr int RTC_MAX_CLK = 16;                   // largest K-split cluster (non-portable size)
 
 template <bool WF32> struct RtcCfg {
     static constexpr int STAGES = WF32 ? 2 : 4;
@@ -253,10 +254,14 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
             const int e = lane + 32 * v;
             float r = 0.f;
             if (e < E) {
-                for (int c = 0; c < CLK; ++c) {
-                    const float *remote = cluster.map_shared_rank(part, c);
-                    r += remote[j * RTC_PART_LD + e];
-                }
+                // all CLK remote loads issued together, summed in rank order
+                float pv[RTC_MAX_CLK];
+#pragma unroll
+                for (int c = 0; c < RTC_MAX_CLK; ++c)
+                    pv[c] = c < CLK ? cluster.map_shared_rank(part, c)[j * RTC_PART_LD + e] : 0.f;
+#pragma unroll
+                for (int c = 0; c < RTC_MAX_CLK; ++c)
+                    if (c < CLK) r += pv[c];
             }
             logit[v] = r;
         }

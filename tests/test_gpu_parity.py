@@ -118,6 +118,8 @@ SMALL = {
     # name: (base config, overrides)
     "bf16_tiles": ("glm5_prefill", dict(N=300, D=512, E=8, k=4, d_moe=384, d_sh=384)),
     "bf16_ragged": ("glm5_prefill", dict(N=257, D=520, E=6, k=3, d_moe=200, d_sh=136)),
+    # more than 2048 (token, slot) ids: the three-kernel dispatch over several chunks
+    "bf16_multichunk": ("glm5_prefill", dict(N=700, D=264, E=12, k=4, d_moe=136, d_sh=200)),
     "bf16_group": ("skew_grouped", dict(N=200, D=256, E=32, n_group=4, topk_group=2, k=4,
                                         d_moe=128, d_sh=256, skew=False)),
     "bf16_single_token": ("glm5_decode", dict(N=1, D=256, E=16, k=8, d_moe=128, d_sh=128)),
