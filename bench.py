@@ -160,6 +160,27 @@ def stored_traffic(kernel: str, workload: str):
         return None
 
 
+# ---- multi-rank host logic (replicas: one independent batch per rank) --------
+def replica_token_seed(rank: int) -> int:
+    """Seed of rank r's token batch: rank 0 keeps the workload's own batch (seed 0
+    draws), every other rank draws a fresh batch so replicas route differently."""
+    return 0 if rank == 0 else 1000 + rank
+
+
+def max_over_ranks(value: float, dist, device) -> float:
+    """Max of a per-rank measurement over all ranks (the job ends with the slowest)."""
+    if dist is None:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tokens_per_s(tokens_per_rank: int, world: int, steps: int, max_ms: float) -> float:
+    """Tokens of all ranks over the slowest rank's time for `steps` steps."""
+    return tokens_per_rank * world * steps / (max_ms / 1e3)
+
+
 def kernel_work(cfg, name: str, hit: int):
     """Algorithmic FLOPs and bytes of one launch (routed k experts, shared expert,
     router; weights of hit experts read once, x read once, y written once)."""
@@ -263,13 +284,13 @@ def main():
     if world > 1:
         import torch.distributed as dist
 
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=60), device_id=dev)
 
     cfg, over = workload(args)
     inp = make_inputs(cfg, seed=0, device=dev)
     if rank > 0:  # each replica gets its own batch of tokens
         from workloads import make_tokens
-        inp.x = make_tokens(cfg, cfg.N, seed=1000 + rank, device=dev)
+        inp.x = make_tokens(cfg, cfg.N, seed=replica_token_seed(rank), device=dev)
     N, D = cfg.N, cfg.D
     ws = torch.empty(max(moe.moe_forward_workspace(N, D, cfg.E, cfg.d_moe, cfg.d_sh, cfg.k,
                                                    cfg.dtype), 256), dtype=torch.uint8, device=dev)
@@ -332,13 +353,9 @@ def main():
     status = moe.moe_device_status(stream)
     if status != 0:
         raise SystemExit("device status after timing: %s" % moe.moe_status_string(status))
-    total_ms = start.elapsed_time(end)
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if dist:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = max_over_ranks(start.elapsed_time(end), dist, dev)
     ms_per_step = total_ms / K
-    value = N * world * K / (total_ms / 1e3)
+    value = whole_job_tokens_per_s(N, world, K, total_ms)
 
     # Per-kernel durations over the timed region.
     per = {"router": sum(evs[s][0].elapsed_time(evs[s][1]) for s in range(K)) / K}
@@ -383,10 +400,7 @@ def main():
         y_host.copy_(y, non_blocking=True)
     e1.record(stream)
     e1.synchronize()
-    et = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-    if dist:
-        dist.all_reduce(et, op=dist.ReduceOp.MAX)
-    e2e_value = N * world * K / (float(et.item()) / 1e3)
+    e2e_value = whole_job_tokens_per_s(N, world, K, max_over_ranks(e0.elapsed_time(e1), dist, dev))
     es = inp.x.element_size()
     clocks = sampler.stop()
 

@@ -48,23 +48,28 @@ def build(force: bool = False) -> str:
     return _LIB
 
 
+def configure(lib):
+    """Declare the C signatures on a loaded oracle library (also used by the tests
+    that load deliberately broken copies of oracle.c)."""
+    P = ctypes.c_void_p
+    I = ctypes.c_int
+    Dd = ctypes.c_double
+    lib.oracle_num_threads.restype = I
+    lib.oracle_router_logits.argtypes = [P, I, P, I, I, I, I, P]
+    lib.oracle_router_logits.restype = None
+    lib.oracle_select.argtypes = [P, P, I, I, I, I, I, I, Dd, P, P, P, P, P, P]
+    lib.oracle_select.restype = I
+    lib.oracle_forward.argtypes = [P, P, P, P, P, P, I, P, P, I, I, I, I, I, I, P, I, P]
+    lib.oracle_forward.restype = I
+    return lib
+
+
 def _load():
     global _lib
     with _lock:
         if _lib is None:
             build()
-            lib = ctypes.CDLL(_LIB)
-            P = ctypes.c_void_p
-            I = ctypes.c_int
-            Dd = ctypes.c_double
-            lib.oracle_num_threads.restype = I
-            lib.oracle_router_logits.argtypes = [P, I, P, I, I, I, I, P]
-            lib.oracle_router_logits.restype = None
-            lib.oracle_select.argtypes = [P, P, I, I, I, I, I, I, Dd, P, P, P, P, P, P]
-            lib.oracle_select.restype = I
-            lib.oracle_forward.argtypes = [P, P, P, P, P, P, I, P, P, I, I, I, I, I, I, P, I, P]
-            lib.oracle_forward.restype = I
-            _lib = lib
+            _lib = configure(ctypes.CDLL(_LIB))
     return _lib
 
 
