@@ -40,11 +40,6 @@ BF16_KERNELS = ["dispatch_count", "dispatch_scan", "dispatch_scatter", "dispatch
                 "gate_up_swiglu", "down_combine_shared"]
 F32_KERNELS = ["dispatch_count", "dispatch_scan", "dispatch_scatter", "gate_up_routed",
                "gate_up_shared", "down_routed", "down_shared", "combine"]
-KERNEL_SOURCES = {
-    "gate_up_swiglu": "sparse_moe_layer_02_b200/csrc/gemm_sm100.cuh",
-    "down_combine_shared": "sparse_moe_layer_02_b200/csrc/gemm_sm100.cuh",
-    "router": "sparse_moe_layer_02_b200/csrc/router.cuh",
-}
 
 
 def parse_args():
@@ -147,16 +142,16 @@ def source_sha(rel: str) -> str:
 
 
 def stored_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch from the committed ncu summary, if the kernel is unchanged."""
+    """DRAM bytes per launch from the committed ncu summary (profiles/traffic.json),
+    or None when there is none or the kernel's source changed since it was taken."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
-            t = json.load(f)
-        rec = t[kernel][workload]
-        if rec.get("source_sha") != source_sha(KERNEL_SOURCES[kernel]):
+            rec = json.load(f)[kernel][workload]
+        if rec.get("source_sha") != source_sha(rec["source"]):
             return None
         return float(rec["bytes_per_launch"])
-    except (OSError, KeyError, ValueError):
+    except (OSError, KeyError, ValueError, TypeError):
         return None
 
 
@@ -374,7 +369,7 @@ def main():
         roof = {"bound": "tensor", "achieved": flops / dur_s / 1e12,
                 "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s"}
     roof["frac"] = roof["achieved"] / roof["peak"] if roof["peak"] else None
-    roof["traffic"] = stored_traffic(dom, cfg.name) if dom in KERNEL_SOURCES else None
+    roof["traffic"] = stored_traffic(dom, cfg.name) if not over else None
     roof["kernel"] = dom
     roof["peak_source"] = peak_src + (" sustained bf16" if roof["bound"] == "tensor" else " copy")
     roof["ms_per_launch"] = per[dom]
