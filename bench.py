@@ -54,6 +54,9 @@ def parse_args():
                     help="target duration of the oracle's CPU-baseline sample")
     ap.add_argument("--set", action="append", default=[], metavar="FIELD=VALUE",
                     help="override a size of the workload (e.g. E=32) for small profiling cases")
+    ap.add_argument("--graph", action="store_true",
+                    help="capture the K timed steps as one CUDA graph and time one replay "
+                         "(default: launch them one by one)")
     return ap.parse_args()
 
 
@@ -315,10 +318,44 @@ def main():
     # Per-step events: router start/end, then moe_forward's kernel boundaries.
     K = args.steps
     nk = len(kernels)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 2)] for _ in range(K)]
+    # external=True: recorded as graph nodes when the steps are captured into a graph
+    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(nk + 2)]
+           for _ in range(K)]
     for row in evs:  # create the underlying CUDA events
         for e in row:
             e.record(stream)
+    torch.cuda.synchronize()
+
+    def timed_steps():
+        st = torch.cuda.current_stream()  # the capture stream while a graph is captured
+        for s_ in range(K):
+            row = evs[s_]
+            row[0].record(st)
+            moe.moe_router(inp.x, inp.W_g, inp.b, cfg.n_group, cfg.topk_group, cfg.k,
+                           cfg.norm_topk_prob, cfg.alpha, idx, w, st)
+            moe.moe_profile_set_events(row[1:])
+            moe.moe_forward(inp.x, inp.gate_up, inp.down, inp.sh_gate, inp.sh_up, inp.sh_down,
+                            idx, w, y, ws, st)
+        moe.moe_profile_set_events([])
+
+    # With --graph the K steps are captured once as a CUDA graph (kernel launches,
+    # their profiling events and all) and replayed once inside the timed region.
+    graph = None
+    launches_per_replay = None
+    if args.graph:
+        try:
+            g = torch.cuda.CUDAGraph()
+            c0 = moe.moe_launch_count()
+            with torch.cuda.graph(g):
+                timed_steps()
+            launches_per_replay = moe.moe_launch_count() - c0
+            g.replay()  # untimed first replay (graph upload), also a warm-up pass
+            torch.cuda.synchronize()
+            graph = g
+        except RuntimeError as exc:  # capture refused: fall back to launching the steps
+            print("graph capture failed, timing launches instead: %s" % exc, file=sys.stderr)
+            moe.moe_profile_set_events([])
+            graph = None
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
@@ -329,18 +366,13 @@ def main():
     sampler.start()
     launches0 = moe.moe_launch_count()
     start.record(stream)
-    for s in range(K):
-        row = evs[s]
-        row[0].record(stream)
-        moe.moe_router(inp.x, inp.W_g, inp.b, cfg.n_group, cfg.topk_group, cfg.k,
-                       cfg.norm_topk_prob, cfg.alpha, idx, w, stream)
-        moe.moe_profile_set_events(row[1:])
-        moe.moe_forward(inp.x, inp.gate_up, inp.down, inp.sh_gate, inp.sh_up, inp.sh_down, idx, w,
-                        y, ws, stream)
+    if graph is not None:
+        graph.replay()
+    else:
+        timed_steps()
     end.record(stream)
     end.synchronize()
-    launches = moe.moe_launch_count() - launches0
-    moe.moe_profile_set_events([])
+    launches = launches_per_replay if graph is not None else moe.moe_launch_count() - launches0
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
@@ -410,6 +442,8 @@ def main():
                "sample": "fp64 oracle router + forward on the first %d tokens of the %d-token "
                          "batch, %d repetitions, %.1f s" % (n, cfg.N, reps, el)}
 
+    used_graph = graph is not None
+    del graph
     if dist:
         dist.barrier()
         dist.destroy_process_group()
@@ -436,6 +470,8 @@ def main():
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": N * D * es,
                 "d2h_bytes_per_step": N * D * es},
         "gpu_launches": int(launches),
+        "timing": "one replay of a CUDA graph of the K steps" if used_graph
+                  else "K steps launched one by one",
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)

@@ -37,7 +37,10 @@ struct Profiler {
     explicit Profiler(cudaStream_t s) : st(s) { mark(); }
     void mark() {
         if (next < g_prof_n && g_prof_events[next])
-            cudaEventRecord(static_cast<cudaEvent_t>(g_prof_events[next]), st);
+            // External records become real event-record nodes when the stream is
+            // being captured into a CUDA graph (plain records only order the capture).
+            cudaEventRecordWithFlags(static_cast<cudaEvent_t>(g_prof_events[next]), st,
+                                     cudaEventRecordExternal);
         ++next;
     }
 };
