@@ -175,9 +175,9 @@ int moe_debug_never_signal(int on);
  *     events[0] on its stream before its first kernel and events[i] right after
  *     its i-th kernel launch (i = 1 .. n-1).  The events are caller-owned
  *     cudaEvent_t handles passed as void*; n = 0 turns recording off.  At most
- *     16 events; MOE_ERR_ARG otherwise.  Records are external
- *     (cudaEventRecordExternal), so under stream capture they become event
- *     nodes of the graph and record on every replay.
+ *     16 events; MOE_ERR_ARG otherwise.  Under stream capture the records are
+ *     external (cudaEventRecordExternal), so they become event nodes of the
+ *     graph and record on every replay.
  *   moe_launch_count: kernels launched by this library in this process so far.
  */
 int moe_profile_set_events(void *const *events, int n);

@@ -34,13 +34,25 @@ int g_prof_n = 0;
 struct Profiler {
     cudaStream_t st;
     int next = 0;
-    explicit Profiler(cudaStream_t s) : st(s) { mark(); }
+    bool capturing = false;
+    explicit Profiler(cudaStream_t s) : st(s) {
+        if (g_prof_n > 0) {
+            cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+            capturing = cudaStreamIsCapturing(st, &cs) == cudaSuccess &&
+                        cs == cudaStreamCaptureStatusActive;
+        }
+        mark();
+    }
     void mark() {
-        if (next < g_prof_n && g_prof_events[next])
-            // External records become real event-record nodes when the stream is
-            // being captured into a CUDA graph (plain records only order the capture).
-            cudaEventRecordWithFlags(static_cast<cudaEvent_t>(g_prof_events[next]), st,
-                                     cudaEventRecordExternal);
+        if (next < g_prof_n && g_prof_events[next]) {
+            cudaEvent_t ev = static_cast<cudaEvent_t>(g_prof_events[next]);
+            // Under stream capture an external record becomes an event-record node of
+            // the graph (a plain record would only order the capture).
+            const cudaError_t e = capturing
+                                      ? cudaEventRecordWithFlags(ev, st, cudaEventRecordExternal)
+                                      : cudaEventRecord(ev, st);
+            if (e != cudaSuccess) cudaGetLastError(); // profiling never fails the call
+        }
         ++next;
     }
 };
