@@ -113,6 +113,21 @@ int moe_forward(const void *x, const void *gate_up, const void *down, const void
                 const float *topk_w, int N, int D, int E, int d_moe, int d_sh, int k,
                 int dtype, void *y, void *workspace, size_t ws_bytes, void *stream);
 
+/*
+ * moe_forward_clamped — moe_forward with the clamped SwiGLU of the
+ * "GLM-5.3-Flash Module 02" page, section 3: every expert, routed or shared,
+ * computes a = min(W_gate x, gate_max) (the gate is clamped from above only),
+ * u = clip(W_up x, -up_max, up_max) and E(x) = W_down (SiLU(a) (.) u).  That
+ * page's model uses gate_max = up_max = 10.  Same arguments, layouts,
+ * workspace and errors as moe_forward; gate_max = up_max = +infinity gives
+ * moe_forward exactly.  MOE_ERR_ARG for a NaN limit or up_max < 0.
+ */
+int moe_forward_clamped(const void *x, const void *gate_up, const void *down,
+                        const void *sh_gate, const void *sh_up, const void *sh_down,
+                        const int32_t *topk_idx, const float *topk_w, int N, int D, int E,
+                        int d_moe, int d_sh, int k, int dtype, float gate_max, float up_max,
+                        void *y, void *workspace, size_t ws_bytes, void *stream);
+
 /* Bytes of device scratch built into the library for moe_forward_noalloc. */
 #define MOE_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
 

@@ -59,7 +59,7 @@ def configure(lib):
     lib.oracle_router_logits.restype = None
     lib.oracle_select.argtypes = [P, P, I, I, I, I, I, I, Dd, P, P, P, P, P, P]
     lib.oracle_select.restype = I
-    lib.oracle_forward.argtypes = [P, P, P, P, P, P, I, P, P, I, I, I, I, I, I, P, I, P]
+    lib.oracle_forward.argtypes = [P, P, P, P, P, P, I, P, P, I, I, I, I, I, I, P, I, Dd, Dd, P]
     lib.oracle_forward.restype = I
     return lib
 
@@ -139,11 +139,14 @@ def router(x: torch.Tensor, W_g: torch.Tensor, b: torch.Tensor, n_group: int, to
     return select(router_logits(x, W_g), b, n_group, topk_group, k, norm_topk_prob, alpha)
 
 
-def forward(x, gate_up, down, sh_gate, sh_up, sh_down, idx, w, tokens=None) -> np.ndarray:
+def forward(x, gate_up, down, sh_gate, sh_up, sh_down, idx, w, tokens=None,
+            gate_max: float = float("inf"), up_max: float = float("inf")) -> np.ndarray:
     """y rows for `tokens` (default all), token-major fp64 (GLM-4.5 MoE Forward, y_n).
 
     x [N,D]; gate_up [E,2d,D]; down [E,D,d]; sh_gate, sh_up [d_sh,D]; sh_down [D,d_sh];
     idx [N,k] (value E = sentinel, skipped); w [N,k] (alpha already included).
+    gate_max / up_max: clamped SwiGLU (GLM-5.3-Flash Module 02, section 3):
+    a = min(gate, gate_max), u = clip(up, -up_max, up_max); infinity = plain SwiGLU.
     """
     x, gate_up, down = _host(x), _host(gate_up), _host(down)
     sh_gate, sh_up, sh_down = _host(sh_gate), _host(sh_up), _host(sh_down)
@@ -167,7 +170,8 @@ def forward(x, gate_up, down, sh_gate, sh_up, sh_down, idx, w, tokens=None) -> n
     y = np.empty((len(tokens), D), dtype=np.float64)
     rc = _load().oracle_forward(_ptr(x), _ptr(gate_up), _ptr(down), _ptr(sh_gate), _ptr(sh_up),
                                 _ptr(sh_down), dt, _ptr(idx), _ptr(w), N, D, E, d, d_sh, k,
-                                _ptr(tokens), len(tokens), _ptr(y))
+                                _ptr(tokens), len(tokens), float(gate_max), float(up_max),
+                                _ptr(y))
     if rc != 0:
         raise ValueError("oracle_forward rejected its arguments (token or expert id out of range)")
     return y

@@ -27,6 +27,11 @@
  *   [SH]  "GLM-5 Shared output", MLP excerpt: the shared expert is
  *         down(silu(gate x) * up x) with gate/up of shape (d_sh, D) and down (D, d_sh),
  *         applied to the same input as the routed experts.
+ *   [CL]  "GLM-5.3-Flash Module 02", section 3: the clamped SwiGLU variant of
+ *         another model, a = min(W_g x, 10) (gate clamped above only),
+ *         u = clip(W_u x, -10, 10), f = W_d (SiLU(a) (.) u), for every expert,
+ *         routed or shared.  Here the limits are parameters (gate_max, up_max);
+ *         +infinity gives the plain SwiGLU of [MF].
  *
  * Readings where the pages are silent (each is listed with its reason in the
  * design notes): discarded groups are masked to -infinity (the zero-fill
@@ -293,13 +298,20 @@ int oracle_router(const void *x, int x_dt, const void *wg, int wg_dt, const floa
 static void swiglu_accumulate(const void *w_gu, size_t gate_base, const void *w_up,
                               size_t up_base, const void *w_down, size_t down_base, int dt,
                               int D, int dd, const double *xn, double scale, double *y,
-                              double *row, double *h)
+                              double *row, double *h, double gate_max, double up_max)
 {
     for (int r = 0; r < dd; ++r) {
         widen_row(w_gu, dt, gate_base + (size_t)r * D, D, row);
         double a = dot(row, xn, D);
         widen_row(w_up, dt, up_base + (size_t)r * D, D, row);
         double u = dot(row, xn, D);
+        /* [CL]: the gate is clamped from above only, the up projection both sides */
+        if (a > gate_max)
+            a = gate_max;
+        if (u > up_max)
+            u = up_max;
+        if (u < -up_max)
+            u = -up_max;
         h[r] = silu(a) * u;
     }
     for (int c = 0; c < D; ++c) {
@@ -316,11 +328,13 @@ static void swiglu_accumulate(const void *w_gu, size_t gate_base, const void *w_
  * w [N,k] double.  tokens[0..n_tokens) lists which rows to evaluate;
  * y [n_tokens, D] double receives them in list order.
  * Indices outside [0, E] are rejected (-1); the sentinel E contributes nothing.
+ * gate_max / up_max: the [CL] limits (+infinity for the plain SwiGLU).
  */
 int oracle_forward(const void *x, const void *gate_up, const void *down, const void *sh_gate,
                    const void *sh_up, const void *sh_down, int dt, const int32_t *idx,
                    const double *w, int N, int D, int E, int d, int d_sh, int k,
-                   const int32_t *tokens, int n_tokens, double *y)
+                   const int32_t *tokens, int n_tokens, double gate_max, double up_max,
+                   double *y)
 {
     for (int t = 0; t < n_tokens; ++t)
         if (tokens[t] < 0 || tokens[t] >= N)
@@ -352,11 +366,11 @@ int oracle_forward(const void *x, const void *gate_up, const void *down, const v
                 const size_t gu = (size_t)i * 2 * (size_t)d * D;
                 swiglu_accumulate(gate_up, gu, gate_up, gu + (size_t)d * D, down,
                                   (size_t)i * D * (size_t)d, dt, D, d, xn,
-                                  w[(size_t)n * k + j], yn, row, h);
+                                  w[(size_t)n * k + j], yn, row, h, gate_max, up_max);
             }
             /* Always-on shared expert, scale 1. */
             swiglu_accumulate(sh_gate, 0, sh_up, 0, sh_down, 0, dt, D, d_sh, xn, 1.0, yn, row,
-                              h);
+                              h, gate_max, up_max);
         }
         free(xn);
         free(row);

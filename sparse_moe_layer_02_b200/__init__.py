@@ -34,7 +34,7 @@ MOE_OK = 0
 EXPORTED_SYMBOLS = ("moe_router", "moe_forward_workspace", "moe_forward", "moe_device_status",
                     "moe_status_string", "moe_version", "moe_debug_set_wait_limit_ns",
                     "moe_debug_never_signal", "moe_profile_set_events", "moe_launch_count",
-                    "moe_forward_noalloc")
+                    "moe_forward_noalloc", "moe_forward_clamped")
 
 
 class MoEError(RuntimeError):
@@ -81,6 +81,9 @@ def load_library():
         lib.moe_launch_count.restype = ctypes.c_ulonglong
         lib.moe_forward_noalloc.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, P, P]
         lib.moe_forward_noalloc.restype = I
+        lib.moe_forward_clamped.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, F, P,
+                                            P, ctypes.c_size_t, P]
+        lib.moe_forward_clamped.restype = I
         _lib = lib
         return lib
 
@@ -149,8 +152,11 @@ def moe_forward_workspace(N: int, D: int, E: int, d_moe: int, d_sh: int, k: int,
 
 
 def moe_forward(x, gate_up, down, sh_gate, sh_up, sh_down, topk_idx, topk_w, y=None,
-                workspace=None, stream=None):
-    """Routed experts + weighted combine + shared expert; returns y [N, D]."""
+                workspace=None, stream=None, gate_max=None, up_max=None):
+    """Routed experts + weighted combine + shared expert; returns y [N, D].
+
+    gate_max / up_max (optional): the clamped SwiGLU (gate clamped from above at
+    gate_max, up clipped to [-up_max, up_max]) via moe_forward_clamped."""
     lib = load_library()
     N, D = x.shape
     E, two_d, D2 = gate_up.shape
@@ -170,12 +176,18 @@ def moe_forward(x, gate_up, down, sh_gate, sh_up, sh_down, topk_idx, topk_w, y=N
     ws_bytes = int(lib.moe_forward_workspace(N, D, E, d, d_sh, k, _dt(x)))
     if workspace is None:
         workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=x.device)
-    rc = lib.moe_forward(_dev(x, "x"), _dev(gate_up, "gate_up"), _dev(down, "down"),
-                         _dev(sh_gate, "sh_gate"), _dev(sh_up, "sh_up"), _dev(sh_down, "sh_down"),
-                         _dev(topk_idx, "topk_idx"), _dev(topk_w, "topk_w"), N, D, E, d, d_sh, k,
-                         _dt(x), _dev(y, "y"), _dev(workspace, "workspace"),
-                         workspace.numel() * workspace.element_size(), _stream(stream))
-    _check(rc, "moe_forward")
+    ptrs = (_dev(x, "x"), _dev(gate_up, "gate_up"), _dev(down, "down"), _dev(sh_gate, "sh_gate"),
+            _dev(sh_up, "sh_up"), _dev(sh_down, "sh_down"), _dev(topk_idx, "topk_idx"),
+            _dev(topk_w, "topk_w"), N, D, E, d, d_sh, k, _dt(x))
+    tail = (_dev(y, "y"), _dev(workspace, "workspace"),
+            workspace.numel() * workspace.element_size(), _stream(stream))
+    if gate_max is None and up_max is None:
+        _check(lib.moe_forward(*ptrs, *tail), "moe_forward")
+    else:
+        inf = float("inf")
+        gm = inf if gate_max is None else float(gate_max)
+        um = inf if up_max is None else float(up_max)
+        _check(lib.moe_forward_clamped(*ptrs, gm, um, *tail), "moe_forward_clamped")
     return y
 
 

@@ -235,4 +235,14 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
 // SiLU(a) = a * sigmoid(a), with the fast exponential.
 __device__ __forceinline__ float silu_f(float a) { return a / (1.0f + __expf(-a)); }
 
+// SwiGLU of one gate/up pair with the optional limits of the clamped variant
+// ("GLM-5.3-Flash Module 02", section 3: the gate is clamped from above only, the
+// up projection on both sides); +infinity limits give the plain SwiGLU.  The
+// comparisons keep a NaN input a NaN.
+__device__ __forceinline__ float swiglu_f(float g, float u, float gate_max, float up_max) {
+    g = g > gate_max ? gate_max : g;
+    u = u > up_max ? up_max : (u < -up_max ? -up_max : u);
+    return silu_f(g) * u;
+}
+
 }  // namespace moe

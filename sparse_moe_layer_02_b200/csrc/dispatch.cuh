@@ -258,49 +258,40 @@ __global__ void __launch_bounds__(DISPATCH_SMALL_THREADS) dispatch_small_kernel(
     }
 }
 
-// Padding rows (beyond an expert's count inside its last tile) carry no
-// token; perm_tok / w_perm are left unset there and every reader checks this.
-__device__ __forceinline__ int expert_of_tile(const int *tile_off, int E, int mt) {
-    int lo = 0, hi = E - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (tile_off[mid] <= mt) lo = mid; else hi = mid - 1;
-    }
-    return lo;
-}
-
-// Copy x[perm_tok[r]] to x_perm[r] for every real permuted row; one warp per row,
-// 16-byte vectors.  row_bytes is a multiple of 16.
+// Copy each token's row of x to its k permuted rows (x_perm[pos_of[n, j]]), one
+// warp per token: the row is read once (x is usually larger than L2, and the
+// permuted order would otherwise re-read each row k times) and written k times,
+// with 16-byte vectors, four per lane in flight.  Padding rows stay unwritten:
+// an MMA output row depends only on its own operand row, and padding rows' outputs
+// are never stored or read.  row_bytes is a multiple of 16.
 __global__ void __launch_bounds__(256) dispatch_gather_kernel(const uint8_t *__restrict__ x,
                                                               uint8_t *__restrict__ x_perm,
                                                               const DispatchParams p,
-                                                              int row_bytes, int rows_max) {
-    __shared__ int s_off[DISPATCH_MAXE + 1];
-    __shared__ int s_cnt[DISPATCH_MAXE];
-    for (int e = threadIdx.x; e <= p.E; e += blockDim.x) {
-        s_off[e] = p.tile_off[e];
-        if (e < p.E) s_cnt[e] = p.counts[e];
-    }
-    __syncthreads();
-    const int rows = min(s_off[p.E] * p.tile_rows, rows_max);
+                                                              int row_bytes) {
     const int lane = threadIdx.x & 31;
-    for (int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < rows;
-         r += (gridDim.x * blockDim.x) >> 5) {
-        const int e = expert_of_tile(s_off, p.E, r / p.tile_rows);
-        if (r - s_off[e] * p.tile_rows >= s_cnt[e]) continue; // padding row
-        const int tok = p.perm_tok[r];
-        const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)tok * row_bytes);
-        uint4 *dst = reinterpret_cast<uint4 *>(x_perm + (size_t)r * row_bytes);
-        const int nvec = row_bytes >> 4;
-        int v = lane;
-        for (; v + 96 < nvec; v += 128) {
-            const uint4 a = src[v], b = src[v + 32], c = src[v + 64], d = src[v + 96];
-            dst[v] = a;
-            dst[v + 32] = b;
-            dst[v + 64] = c;
-            dst[v + 96] = d;
+    const int nvec = row_bytes >> 4;
+    for (int n = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; n < p.N;
+         n += (gridDim.x * blockDim.x) >> 5) {
+        const int my_pos = lane < p.k ? p.pos_of[(size_t)n * p.k + lane] : -1;
+        const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)n * row_bytes);
+        for (int v0 = 0; v0 < nvec; v0 += 128) {
+            uint4 r[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int v = v0 + lane + 32 * u;
+                if (v < nvec) r[u] = src[v];
+            }
+            for (int j = 0; j < p.k; ++j) {
+                const int pos = __shfl_sync(0xffffffffu, my_pos, j);
+                if (pos < 0) continue;
+                uint4 *dst = reinterpret_cast<uint4 *>(x_perm + (size_t)pos * row_bytes);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int v = v0 + lane + 32 * u;
+                    if (v < nvec) dst[v] = r[u];
+                }
+            }
         }
-        for (; v < nvec; v += 32) dst[v] = src[v];
     }
 }
 

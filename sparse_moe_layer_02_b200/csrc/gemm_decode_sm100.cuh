@@ -62,6 +62,7 @@ struct DecArgs {
     const __nv_bfloat16 *slot;
     uint64_t wait_limit_ns;
     int never_signal;
+    float gate_max, up_max; // gate_up: SwiGLU limits (+infinity = plain SwiGLU)
 };
 
 struct DecTile {
@@ -308,8 +309,9 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
                             uint32_t pk[4];
 #pragma unroll
                             for (int h = 0; h < 4; ++h)
-                                pk[h] = pack_bf16x2(silu_f(g[2 * h]) * u[2 * h],
-                                                    silu_f(g[2 * h + 1]) * u[2 * h + 1]);
+                                pk[h] = pack_bf16x2(swiglu_f(g[2 * h], u[2 * h], a.gate_max, a.up_max),
+                                                    swiglu_f(g[2 * h + 1], u[2 * h + 1], a.gate_max,
+                                                             a.up_max));
                             *reinterpret_cast<uint4 *>(out + (size_t)(c.row0 + tk) * ld + col) =
                                 make_uint4(pk[0], pk[1], pk[2], pk[3]);
                         }

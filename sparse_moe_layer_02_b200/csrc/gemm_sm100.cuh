@@ -69,6 +69,7 @@ struct GemmArgs {
     float *osh;                // down: shared expert output [N, ld_s] fp32
     uint64_t wait_limit_ns;
     int never_signal;
+    float gate_max, up_max; // gate_up: SwiGLU limits (+infinity = plain SwiGLU)
 };
 
 struct TileCoord {
@@ -375,7 +376,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                         float h[32];
 #pragma unroll
                         for (int i = 0; i < 32; ++i)
-                            h[i] = silu_f(__uint_as_float(g[i])) * __uint_as_float(u[i]);
+                            h[i] = swiglu_f(__uint_as_float(g[i]), __uint_as_float(u[i]),
+                                            a.gate_max, a.up_max);
                         store_row_chunk_bf16(row_ptr, col, ncols, h);
                     }
                 }

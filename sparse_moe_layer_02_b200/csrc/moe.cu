@@ -459,10 +459,16 @@ size_t moe_forward_workspace(int N, int D, int E, int d_moe, int d_sh, int k, in
     return L.total;
 }
 
-int moe_forward(const void *x, const void *gate_up, const void *down, const void *sh_gate,
-                const void *sh_up, const void *sh_down, const int32_t *topk_idx,
-                const float *topk_w, int N, int D, int E, int d_moe, int d_sh, int k, int dtype,
-                void *y, void *workspace, size_t ws_bytes, void *stream) {
+}  // extern "C"
+
+namespace moe {
+namespace {
+
+int forward_impl(const void *x, const void *gate_up, const void *down, const void *sh_gate,
+                 const void *sh_up, const void *sh_down, const int32_t *topk_idx,
+                 const float *topk_w, int N, int D, int E, int d_moe, int d_sh, int k, int dtype,
+                 float gate_max, float up_max, void *y, void *workspace, size_t ws_bytes,
+                 void *stream) {
     if (dtype != MOE_F32 && dtype != MOE_BF16) return MOE_ERR_DTYPE;
     if (N < 0 || D <= 0 || E <= 0 || E > DISPATCH_MAXE || d_moe <= 0 || d_sh <= 0 || k <= 0 ||
         k > 32)
@@ -541,6 +547,8 @@ int moe_forward(const void *x, const void *gate_up, const void *down, const void
         a.d = d_moe;
         a.d_sh = d_sh;
         a.k = k;
+        a.gate_max = gate_max;
+        a.up_max = up_max;
         const int rblocks = (int)(L.rows_max / SIMT_T);
         const int nblocks = (N + SIMT_T - 1) / SIMT_T;
         simt_expert_kernel<SIMT_GATEUP_R><<<dim3(rblocks, (d_moe + 31) / 32), 256, 0, st>>>(a);
@@ -560,10 +568,9 @@ int moe_forward(const void *x, const void *gate_up, const void *down, const void
     // ---- bf16 tensor-core path ----
     uint8_t *x_perm = ws + L.x_perm;
     {
-        const int rows = (int)L.rows_max;
-        const int grid = std::min((rows + 7) / 8, dev->sms * 16);
+        const int grid = std::min((N + 7) / 8, dev->sms * 16);
         dispatch_gather_kernel<<<grid, 256, 0, st>>>(static_cast<const uint8_t *>(x), x_perm, dp,
-                                                    D * 2, rows);
+                                                    D * 2);
         if ((rc = launched(prof)) != MOE_OK) return rc;
     }
     __nv_bfloat16 *h_perm = reinterpret_cast<__nv_bfloat16 *>(ws + L.h_perm);
@@ -594,6 +601,8 @@ int moe_forward(const void *x, const void *gate_up, const void *down, const void
         g.tt_s = (N + DEC_TT - 1) / DEC_TT;
         g.wait_limit_ns = g_wait_limit_ns;
         g.never_signal = g_never_signal;
+        g.gate_max = gate_max;
+        g.up_max = up_max;
         // gate_up + SwiGLU: 64 features x 32 tokens per tile
         g.nb_r = (d_moe + 63) / 64;
         g.nb_s = (d_sh + 63) / 64;
@@ -652,6 +661,8 @@ int moe_forward(const void *x, const void *gate_up, const void *down, const void
     g.mt_s = mt_s;
     g.wait_limit_ns = g_wait_limit_ns;
     g.never_signal = g_never_signal;
+    g.gate_max = gate_max;
+    g.up_max = up_max;
 
     // gate_up + SwiGLU
     g.nb_r = (d_moe + 127) / 128;
@@ -692,6 +703,29 @@ int moe_forward(const void *x, const void *gate_up, const void *down, const void
                                 true, st);
     prof.mark();
     return rc;
+}
+
+}  // namespace
+}  // namespace moe
+
+extern "C" {
+
+int moe_forward(const void *x, const void *gate_up, const void *down, const void *sh_gate,
+                const void *sh_up, const void *sh_down, const int32_t *topk_idx,
+                const float *topk_w, int N, int D, int E, int d_moe, int d_sh, int k, int dtype,
+                void *y, void *workspace, size_t ws_bytes, void *stream) {
+    return forward_impl(x, gate_up, down, sh_gate, sh_up, sh_down, topk_idx, topk_w, N, D, E,
+                        d_moe, d_sh, k, dtype, INFINITY, INFINITY, y, workspace, ws_bytes, stream);
+}
+
+int moe_forward_clamped(const void *x, const void *gate_up, const void *down, const void *sh_gate,
+                        const void *sh_up, const void *sh_down, const int32_t *topk_idx,
+                        const float *topk_w, int N, int D, int E, int d_moe, int d_sh, int k,
+                        int dtype, float gate_max, float up_max, void *y, void *workspace,
+                        size_t ws_bytes, void *stream) {
+    if (gate_max != gate_max || up_max != up_max || up_max < 0.f) return MOE_ERR_ARG;
+    return forward_impl(x, gate_up, down, sh_gate, sh_up, sh_down, topk_idx, topk_w, N, D, E,
+                        d_moe, d_sh, k, dtype, gate_max, up_max, y, workspace, ws_bytes, stream);
 }
 
 int moe_device_status(void *stream) {

@@ -1,7 +1,7 @@
 // fp32 expert path on CUDA cores (no TF32: fp32 products and fp32 accumulation),
 // for fp32 layers such as the tiny fully-fp32 configuration.  Same dispatch and
 // same arithmetic as the tensor-core path ("GLM-4.5 MoE Forward", How it works):
-//   gate_up  h[r, c]  = SiLU(x_r . W_gate[c]) * (x_r . W_up[c])   (fp32 h)
+//   gate_up  h[r, c]  = SiLU(x_r . W_gate[c]) * (x_r . W_up[c])   (fp32 h, optional limits)
 //   down     slot[r]  = w_r * (h_r . W_down rows)                 (fp32 slot)
 //            y[n]     = (h_sh . W_sh_down rows)                    (shared, into y)
 //   combine  y[n]    <- sum_j slot[pos(n, j)] + y[n]               (slot order)
@@ -22,6 +22,7 @@ struct SimtArgs {
     const float *w_perm;
     float *h_perm, *h_sh, *slot, *y;
     int N, D, E, d, d_sh, k;
+    float gate_max, up_max; // SwiGLU limits (+infinity = plain SwiGLU)
 };
 
 __device__ __forceinline__ int expert_of_row(const int32_t *tile_off, int E, int row) {
@@ -118,9 +119,9 @@ __global__ void __launch_bounds__(256) simt_expert_kernel(const SimtArgs a) {
             const int c = c0 + tx + 16 * j;
             if (c >= ncols) continue;
             if (MODE == SIMT_GATEUP_R) {
-                a.h_perm[(size_t)r * a.d + c] = silu_f(g[i][j]) * u[i][j];
+                a.h_perm[(size_t)r * a.d + c] = swiglu_f(g[i][j], u[i][j], a.gate_max, a.up_max);
             } else if (MODE == SIMT_GATEUP_S) {
-                a.h_sh[(size_t)r * a.d_sh + c] = silu_f(g[i][j]) * u[i][j];
+                a.h_sh[(size_t)r * a.d_sh + c] = swiglu_f(g[i][j], u[i][j], a.gate_max, a.up_max);
             } else if (MODE == SIMT_DOWN_R) {
                 if (r < seg_end) a.slot[(size_t)r * a.D + c] = a.w_perm[r] * g[i][j];
             } else {

@@ -159,6 +159,31 @@ def test_forward_parity_small(case):
     assert err2["max_rel"] <= Y_TOL[cfg.dtype]
 
 
+@pytest.mark.parametrize("case", ["bf16_prefill", "bf16_decode", "fp32"])
+def test_clamped_swiglu_parity(case):
+    # Clamped SwiGLU of the GLM-5.3-Flash Module 02 page (gate <= 10, |up| <= 10) on
+    # weights scaled so that many projections cross the limits on both sides.
+    base, over = {"bf16_prefill": ("glm5_prefill", dict(N=300, D=512, E=8, k=4, d_moe=256, d_sh=256)),
+                  "bf16_decode": ("glm5_decode", dict(N=64, D=512, E=16, k=4, d_moe=192, d_sh=128)),
+                  "fp32": ("tiny_fp32", dict())}[case]
+    cfg = CONFIGS[base].with_(**over)
+    inp = make_inputs(cfg, seed=31)
+    scale = 40.0 if cfg.D <= 256 else 25.0
+    inp.gate_up = (inp.gate_up.float() * scale).to(cfg.dtype)
+    inp.sh_gate = (inp.sh_gate.float() * scale).to(cfg.dtype)
+    inp.sh_up = (inp.sh_up.float() * scale).to(cfg.dtype)
+    orc = _oracle_route(cfg, inp)
+    y_ref = oracle.forward(*_weights(inp), orc["idx"], orc["w"], gate_max=10.0, up_max=10.0)
+    y_plain = oracle.forward(*_weights(inp), orc["idx"], orc["w"])
+    assert rel_err(y_plain, y_ref)["max_rel"] > 0.05  # the limits really bite
+    d = inp.to(DEV)
+    y = moe.moe_forward(*_weights(d), torch.from_numpy(orc["idx"]).to(DEV),
+                        torch.from_numpy(orc["w"]).float().to(DEV), gate_max=10.0, up_max=10.0)
+    assert moe.moe_device_status() == 0
+    err = rel_err(y.float().cpu().numpy(), y_ref)
+    assert err["finite"] and err["max_rel"] <= Y_TOL[cfg.dtype], err
+
+
 @pytest.mark.parametrize("N", [200, 400])
 def test_forward_sentinel_and_hot_expert(N):
     cfg = CONFIGS["glm5_prefill"].with_(N=N, D=256, E=8, k=4, d_moe=128, d_sh=128)

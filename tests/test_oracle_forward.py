@@ -68,6 +68,51 @@ def test_selection_matrix_experts_closed_form():
     np.testing.assert_allclose(y, expect.numpy(), rtol=1e-14, atol=1e-15)
 
 
+def test_clamped_swiglu_boundaries_closed_form():
+    # "GLM-5.3-Flash Module 02", section 3: a = min(W_g x, 10) (above only),
+    # u = clip(W_u x, -10, 10).  Gate rows pick x[r], up rows pick 1.5 x[r+1]; the
+    # values straddle both limits on both projections, and a gate value of -30 must
+    # stay -30 (a symmetric clamp would give -10, a visibly different SiLU).
+    D, d, E = 6, 4, 1
+    gate_up = torch.zeros(E, 2 * d, D)
+    down = torch.zeros(E, D, d)
+    for r in range(d):
+        gate_up[0, r, r] = 1.0
+        gate_up[0, d + r, r + 1] = 1.5
+        down[0, r, r] = 1.0
+    x = torch.tensor([[15.0, -30.0, 12.0, -20.0, 5.0, 8.0],
+                      [9.5, 6.0, -11.0, 7.0, 10.5, -3.0],
+                      [-30.0, 2.0, 10.0, -7.0, 0.5, 4.0]])
+    sh = dict(sh_gate=torch.zeros(1, D), sh_up=torch.zeros(1, D), sh_down=torch.zeros(D, 1))
+    idx = np.zeros((3, 1), dtype=np.int32)
+    w = np.ones((3, 1))
+    y = oracle.forward(x, gate_up, down, idx=idx, w=w, gate_max=10.0, up_max=10.0, **sh)
+    xd = x.double()
+    a = torch.clamp(xd[:, :d], max=10.0)
+    u = torch.clamp(1.5 * xd[:, 1:d + 1], min=-10.0, max=10.0)
+    expect = torch.zeros(3, D, dtype=torch.float64)
+    expect[:, :d] = F.silu(a) * u
+    np.testing.assert_allclose(y, expect.numpy(), rtol=1e-14, atol=1e-300)
+    # no limits: the plain SwiGLU of the same selection matrices
+    y0 = oracle.forward(x, gate_up, down, idx=idx, w=w, **sh)
+    plain = torch.zeros(3, D, dtype=torch.float64)
+    plain[:, :d] = F.silu(xd[:, :d]) * 1.5 * xd[:, 1:d + 1]
+    np.testing.assert_allclose(y0, plain.numpy(), rtol=1e-14)
+    assert not np.allclose(y, y0)
+
+
+def test_clamp_applies_to_the_shared_expert_too():
+    t = _small(seed=21)
+    t = {k_: (v * 40.0 if k_ != "x" else v) for k_, v in t.items()}  # large activations
+    t["down"] = torch.zeros_like(t["down"])
+    idx, w = _routing(10, 6, 2, 22)
+    y = oracle.forward(**t, idx=idx, w=w, gate_max=10.0, up_max=10.0)
+    x, g, u_, dn = (v.double() for v in (t["x"], t["sh_gate"], t["sh_up"], t["sh_down"]))
+    a = torch.clamp(F.linear(x, g), max=10.0)
+    u = torch.clamp(F.linear(x, u_), -10.0, 10.0)
+    np.testing.assert_allclose(y, F.linear(F.silu(a) * u, dn).numpy(), rtol=1e-12, atol=1e-12)
+
+
 def test_shared_expert_alone_is_the_swiglu_mlp():
     t = _small()
     t["down"] = torch.zeros_like(t["down"])  # routed experts contribute nothing

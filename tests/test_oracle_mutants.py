@@ -42,9 +42,13 @@ MUTANTS = {
                               "if (0) swiglu_accumulate(sh_gate, 0, sh_up, 0, sh_down, 0, dt, D, d_sh, xn, 1.0, yn, row,"),
     "shared_expert_scaled": ("swiglu_accumulate(sh_gate, 0, sh_up, 0, sh_down, 0, dt, D, d_sh, xn, 1.0, yn, row,",
                              "swiglu_accumulate(sh_gate, 0, sh_up, 0, sh_down, 0, dt, D, d_sh, xn, 2.5, yn, row,"),
-    "routed_weight_ignored": ("w[(size_t)n * k + j], yn, row, h);", "1.0, yn, row, h);"),
+    "routed_weight_ignored": ("w[(size_t)n * k + j], yn, row, h, gate_max, up_max);",
+                              "1.0, yn, row, h, gate_max, up_max);"),
     "sentinel_not_skipped": ("const int i = idx[(size_t)n * k + j];\n                if (i == E)",
                              "const int i = idx[(size_t)n * k + j] == E ? E - 1 : idx[(size_t)n * k + j];\n                if (i == E)"),
+    "gate_clamped_both_sides": ("if (a > gate_max)\n            a = gate_max;",
+                                "if (a > gate_max)\n            a = gate_max;\n        if (a < -gate_max)\n            a = -gate_max;"),
+    "up_clamped_above_only": ("if (u < -up_max)\n            u = -up_max;", ""),
     "bf16_widened_wrong": ("uint32_t bits = ((uint32_t)((const uint16_t *)base)[i]) << 16;",
                            "uint32_t bits = ((uint32_t)((const uint16_t *)base)[i]) << 15;"),
 }
