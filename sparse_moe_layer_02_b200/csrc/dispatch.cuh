@@ -258,23 +258,27 @@ __global__ void __launch_bounds__(DISPATCH_SMALL_THREADS) dispatch_small_kernel(
     }
 }
 
-// Copy each token's row of x to its k permuted rows (x_perm[pos_of[n, j]]), one
-// warp per token: the row is read once (x is usually larger than L2, and the
-// permuted order would otherwise re-read each row k times) and written k times,
-// with 16-byte vectors, four per lane in flight.  Padding rows stay unwritten:
-// an MMA output row depends only on its own operand row, and padding rows' outputs
-// are never stored or read.  row_bytes is a multiple of 16.
+// Copy each token's row of x to its k permuted rows (x_perm[pos_of[n, j]]).  A
+// warp takes one 2 KiB piece of one token's row: the piece is read once (x is
+// usually larger than L2, and the permuted order would otherwise re-read each row
+// k times) and written k times, with 16-byte vectors, four per lane in flight.
+// Padding rows stay unwritten: an MMA output row depends only on its own operand
+// row, and padding rows' outputs are never stored or read.  row_bytes is a
+// multiple of 16.
 __global__ void __launch_bounds__(256) dispatch_gather_kernel(const uint8_t *__restrict__ x,
                                                               uint8_t *__restrict__ x_perm,
                                                               const DispatchParams p,
                                                               int row_bytes) {
     const int lane = threadIdx.x & 31;
     const int nvec = row_bytes >> 4;
-    for (int n = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; n < p.N;
-         n += (gridDim.x * blockDim.x) >> 5) {
+    const int pieces = (nvec + 127) / 128;
+    for (int item = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; item < p.N * pieces;
+         item += (gridDim.x * blockDim.x) >> 5) {
+        const int n = item / pieces;
+        const int v0 = (item - n * pieces) * 128;
         const int my_pos = lane < p.k ? p.pos_of[(size_t)n * p.k + lane] : -1;
         const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)n * row_bytes);
-        for (int v0 = 0; v0 < nvec; v0 += 128) {
+        {
             uint4 r[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {

@@ -568,7 +568,8 @@ int forward_impl(const void *x, const void *gate_up, const void *down, const voi
     // ---- bf16 tensor-core path ----
     uint8_t *x_perm = ws + L.x_perm;
     {
-        const int grid = std::min((N + 7) / 8, dev->sms * 16);
+        const int items = N * ((D * 2 / 16 + 127) / 128); // 2 KiB pieces of token rows
+        const int grid = std::min((items + 7) / 8, dev->sms * 16);
         dispatch_gather_kernel<<<grid, 256, 0, st>>>(static_cast<const uint8_t *>(x), x_perm, dp,
                                                     D * 2);
         if ((rc = launched(prof)) != MOE_OK) return rc;
