@@ -314,6 +314,10 @@ def main():
     loads = torch.bincount(idx.flatten().long(), minlength=cfg.E)
     hit = int((loads > 0).sum().item())
     max_over_mean = float(loads.max().item() / loads.float().mean().item())
+    # Routing collisions: (token, expert) pairs served per distinct expert whose
+    # weights the step streams, and the routed weight bytes fetched per token.
+    reuse = float(loads.sum().item()) / max(hit, 1)
+    routed_bytes_per_token = hit * 3.0 * cfg.D * cfg.d_moe * inp.gate_up.element_size() / cfg.N
 
     # Per-step events: router start/end, then moe_forward's kernel boundaries.
     K = args.steps
@@ -459,6 +463,7 @@ def main():
                    "d_moe": cfg.d_moe, "d_sh": cfg.d_sh, "alpha": cfg.alpha,
                    "router_dtype": str(cfg.wg_dtype).replace("torch.", ""),
                    "hit_experts": hit, "max_over_mean_load": max_over_mean,
+                   "reuse_factor": reuse, "routed_weight_bytes_per_token": routed_bytes_per_token,
                    "overrides": over or None,
                    "parallelism": "replicas" if world > 1 else "single",
                    "l2": "inputs larger than L2 (hit-expert weights %.2f GB per step)"

@@ -122,6 +122,23 @@ def test_shared_expert_alone_is_the_swiglu_mlp():
     np.testing.assert_allclose(y, expect.numpy(), rtol=1e-12, atol=1e-14)
 
 
+@pytest.mark.parametrize("n_shared", [2, 3])
+def test_n_shared_experts_are_one_wider_mlp(n_shared):
+    # "GLM-4.5 MoE Forward", How it works: the shared expert is one SwiGLU of
+    # intermediate width d_moe * n_shared.  Its features are independent until
+    # the down projection sums them, so the wide MLP must equal the sum of the
+    # n_shared width-d_moe MLPs cut from its gate/up rows and down columns.
+    d = 8
+    t = _small(d=d, d_sh=d * n_shared, seed=31 + n_shared)
+    idx, w = _routing(10, 6, 2, 32)
+    y = oracle.forward(**t, idx=idx, w=w)
+    zero = {k_: torch.zeros_like(v) for k_, v in t.items() if k_.startswith("sh_")}
+    routed = oracle.forward(t["x"], t["gate_up"], t["down"], idx=idx, w=w, **zero)
+    parts = sum(_lib_swiglu(t["x"], t["sh_gate"][j * d:(j + 1) * d], t["sh_up"][j * d:(j + 1) * d],
+                            t["sh_down"][:, j * d:(j + 1) * d]).numpy() for j in range(n_shared))
+    np.testing.assert_allclose(y, routed + parts, rtol=1e-12, atol=1e-13)
+
+
 def test_routed_expert_matches_library_swiglu():
     t = _small(E=3, N=4)
     sh = dict(sh_gate=torch.zeros_like(t["sh_gate"]), sh_up=t["sh_up"], sh_down=t["sh_down"])
