@@ -42,6 +42,8 @@ MUTANTS = {
                               "if (0) swiglu_accumulate(sh_gate, 0, sh_up, 0, sh_down, 0, dt, D, d_sh, xn, 1.0, yn, row,"),
     "shared_expert_scaled": ("swiglu_accumulate(sh_gate, 0, sh_up, 0, sh_down, 0, dt, D, d_sh, xn, 1.0, yn, row,",
                              "swiglu_accumulate(sh_gate, 0, sh_up, 0, sh_down, 0, dt, D, d_sh, xn, 2.5, yn, row,"),
+    "shared_width_capped_at_d_moe": ("swiglu_accumulate(sh_gate, 0, sh_up, 0, sh_down, 0, dt, D, d_sh, xn, 1.0,",
+                                     "swiglu_accumulate(sh_gate, 0, sh_up, 0, sh_down, 0, dt, D, d_sh < d ? d_sh : d, xn, 1.0,"),
     "routed_weight_ignored": ("w[(size_t)n * k + j], yn, row, h, gate_max, up_max);",
                               "1.0, yn, row, h, gate_max, up_max);"),
     "sentinel_not_skipped": ("const int i = idx[(size_t)n * k + j];\n                if (i == E)",
