@@ -44,21 +44,21 @@ __host__ __device__ constexpr int router_smem_bytes(int EV) {
             (ROUTER_THREADS / 32) * ROUTER_MAXV * 32) * 4;
 }
 
-// (value, index) comparison: larger value wins, ties go to the lower index.
-__device__ __forceinline__ bool better(float v, int i, float bv, int bi) {
-    return v > bv || (v == bv && i < bi);
+// Unsigned key with the order of the floats: a larger float has a larger key
+// (-inf included, -0 equal to +0); NaN maps to 0, below every number, so it is
+// never preferred to a number.
+__device__ __forceinline__ uint32_t order_key(float v) {
+    if (v != v) return 0u;
+    const uint32_t b = __float_as_uint(v == 0.f ? 0.f : v);
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
-__device__ __forceinline__ void warp_argmax(float &v, int &i) {
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-        float ov = __shfl_xor_sync(0xffffffffu, v, off);
-        int oi = __shfl_xor_sync(0xffffffffu, i, off);
-        if (better(ov, oi, v, i)) {
-            v = ov;
-            i = oi;
-        }
-    }
+// Warp-wide pick of the best (key, id) pair: the largest key, and among the lanes
+// holding it the smallest id.  Lanes with nothing to offer pass key 0 and id
+// 0xffffffff.  Two redux.sync reductions instead of a shuffle butterfly.
+__device__ __forceinline__ uint32_t warp_pick(uint32_t key, uint32_t id) {
+    const uint32_t m = __reduce_max_sync(0xffffffffu, key);
+    return __reduce_min_sync(0xffffffffu, key == m ? id : 0xffffffffu);
 }
 
 // Selection for one token by one warp ("GLM-4.5 Group Router", How it works):
@@ -111,19 +111,19 @@ __device__ __forceinline__ void router_select(const RouterParams &p, int t, cons
         }
         __syncwarp();
         uint64_t kept = 0;
+        const uint32_t gk[2] = {order_key(gs[0]), order_key(gs[1])};
         for (int r = 0; r < p.tg; ++r) {
-            float bv = -INFINITY;
-            int bi = 0x7fffffff;
+            uint32_t bk = 0, bi = 0xffffffffu;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const int g = lane + 32 * h;
-                if (g < G && !((kept >> g) & 1ull) && better(gs[h], g, bv, bi)) {
-                    bv = gs[h];
+                if (g < G && !((kept >> g) & 1ull) && (bi == 0xffffffffu || gk[h] > bk)) {
+                    bk = gk[h];
                     bi = g;
                 }
             }
-            warp_argmax(bv, bi);
-            kept |= 1ull << bi;
+            const uint32_t win = warp_pick(bk, bi);
+            if (win < 64u) kept |= 1ull << win;
         }
 #pragma unroll
         for (int v = 0; v < EV; ++v) {
@@ -135,24 +135,24 @@ __device__ __forceinline__ void router_select(const RouterParams &p, int t, cons
         for (int v = 0; v < EV; ++v)
             if (lane + 32 * v < E) cand |= 1u << v;
     }
-    // Top-k by s' among candidates; lane r keeps the r-th pick.
+    // Top-k by s' among candidates; lane r keeps the r-th pick.  A lane's own
+    // experts rise with v, so its first maximal key is its smallest id.
+    uint32_t key[EV];
+#pragma unroll
+    for (int v = 0; v < EV; ++v) key[v] = order_key(sp[v]);
     int my_e = -1;
     float my_s = 0.f;
     for (int r = 0; r < p.k; ++r) {
-        float bv = -INFINITY;
-        int bi = 0x7fffffff;
+        uint32_t bk = 0, bi = 0xffffffffu;
 #pragma unroll
         for (int v = 0; v < EV; ++v) {
-            if ((cand >> v) & 1u) {
-                const int e = lane + 32 * v;
-                if (better(sp[v], e, bv, bi)) {
-                    bv = sp[v];
-                    bi = e;
-                }
+            if (((cand >> v) & 1u) && (bi == 0xffffffffu || key[v] > bk)) {
+                bk = key[v];
+                bi = lane + 32 * v;
             }
         }
-        warp_argmax(bv, bi);
-        const int owner = bi & 31, vw = bi >> 5;
+        const int win = (int)warp_pick(bk, bi);
+        const int owner = win & 31, vw = win >> 5;
         float sv = 0.f;
 #pragma unroll
         for (int v = 0; v < EV; ++v)
@@ -160,7 +160,7 @@ __device__ __forceinline__ void router_select(const RouterParams &p, int t, cons
         sv = __shfl_sync(0xffffffffu, sv, owner);
         if (lane == owner) cand &= ~(1u << vw);
         if (lane == r) {
-            my_e = bi;
+            my_e = win;
             my_s = sv;
         }
     }

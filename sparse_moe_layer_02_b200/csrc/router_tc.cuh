@@ -182,39 +182,55 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
         }
         __syncwarp();
     } else if (WF32) {
-        // Split fp32 W_g into three bf16 tiles per stage (warps 2-7).
+        // Split fp32 W_g into three bf16 tiles per stage (warps 2-7).  A thread owns
+        // up to SPLIT_IT 8-float pieces of a k-block.  The next k-block's pieces are
+        // loaded into registers while the current ones are split and stored, so the
+        // load latency is paid once per k-block rather than once per piece.
+        constexpr int SPLIT_IT = (RTC_MAXE_F32 * 8 + NCONV * 32 - 1) / (NCONV * 32);
         const int cw = warp - 2, ct = cw * 32 + lane;
         const float *W = static_cast<const float *>(p.W_g);
+        float4 ru[SPLIT_IT], rv[SPLIT_IT];
+        auto fetch = [&](int kb) {
+            const int k0 = kb * RTC_BK;
+#pragma unroll
+            for (int j = 0; j < SPLIT_IT; ++j) {
+                const int item = ct + j * NCONV * 32;
+                ru[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+                rv[j] = ru[j];
+                if (item < E * 8) {
+                    const int row = item >> 3, kk = k0 + (item & 7) * 8;
+                    const float *src = W + (size_t)row * p.D + kk;
+                    if (kk + 8 <= p.D) {
+                        ru[j] = __ldg(reinterpret_cast<const float4 *>(src));
+                        rv[j] = __ldg(reinterpret_cast<const float4 *>(src) + 1);
+                    } else {
+                        float t[8];
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) t[q] = kk + q < p.D ? src[q] : 0.f;
+                        ru[j] = make_float4(t[0], t[1], t[2], t[3]);
+                        rv[j] = make_float4(t[4], t[5], t[6], t[7]);
+                    }
+                }
+            }
+        };
+        if (nkb > 0) fetch(kb_of(0));
         uint32_t it = 0;
         for (int i = 0; i < nkb; ++i, ++it) {
-            const int kb = kb_of(i);
             const uint32_t s = it % C::STAGES, ph = (it / C::STAGES) & 1;
             bool ok = true;
             if (lane == 0) ok = mbar_wait(&empty[s], ph ^ 1, limit, abort_flag, 330);
             ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
             if (!ok) break;
             uint8_t *b0 = ring + s * C::STAGE_BYTES + RTC_A_BYTES;
-            const int k0 = kb * RTC_BK;
-            for (int item = ct; item < E * 8; item += NCONV * 32) {
-                const int row = item >> 3, chunk = item & 7;
-                const int kk = k0 + chunk * 8;
-                float4 u = make_float4(0.f, 0.f, 0.f, 0.f), v = u;
-                const float *src = W + (size_t)row * p.D + kk;
-                if (kk + 8 <= p.D) {
-                    u = __ldg(reinterpret_cast<const float4 *>(src));
-                    v = __ldg(reinterpret_cast<const float4 *>(src) + 1);
-                } else {
-                    float t[8];
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) t[q] = kk + q < p.D ? src[q] : 0.f;
-                    u = make_float4(t[0], t[1], t[2], t[3]);
-                    v = make_float4(t[4], t[5], t[6], t[7]);
-                }
-                split_store(b0, row, chunk, u, v, C::B_PART);
+            for (int j = 0; j < SPLIT_IT; ++j) {
+                const int item = ct + j * NCONV * 32;
+                if (item < E * 8) split_store(b0, item >> 3, item & 7, ru[j], rv[j], C::B_PART);
             }
             fence_proxy_async_smem(); // generic-proxy stores -> visible to the tensor core
             __syncwarp();
             if (lane == 0) mbar_arrive(&full[s]);
+            if (i + 1 < nkb) fetch(kb_of(i + 1));
         }
         __syncwarp();
     }
@@ -243,27 +259,36 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
     cluster.sync();
 
     // ---- sum the cluster's partial logits and select: one warp per token -------
-    const int tpc = RTC_BM / CLK; // tokens finalised by this CTA
-    for (int jl = warp; jl < tpc; jl += RTC_THREADS / 32) {
-        const int j = rank * tpc + jl;
+    // Token j of the block goes to CTA j % CLK, so a small batch spreads over the
+    // whole cluster.  A lane loads the partials of its experts from every CTA of
+    // the cluster (VB expert slots x CLK ranks in flight) before it adds any, and
+    // adds them in rank order (deterministic).
+    constexpr int VB = EV < 4 ? EV : 4;
+    for (int jl = warp; rank + CLK * jl < RTC_BM; jl += RTC_THREADS / 32) {
+        const int j = rank + CLK * jl;
         const int t = t0 + j;
         if (t >= p.N) break;
         float logit[EV];
 #pragma unroll
-        for (int v = 0; v < EV; ++v) {
-            const int e = lane + 32 * v;
-            float r = 0.f;
-            if (e < E) {
-                // all CLK remote loads issued together, summed in rank order
-                float pv[RTC_MAX_CLK];
+        for (int v0 = 0; v0 < EV; v0 += VB) {
+            float pv[VB][RTC_MAX_CLK];
 #pragma unroll
-                for (int c = 0; c < RTC_MAX_CLK; ++c)
-                    pv[c] = c < CLK ? cluster.map_shared_rank(part, c)[j * RTC_PART_LD + e] : 0.f;
+            for (int c = 0; c < RTC_MAX_CLK; ++c) {
+                const float *src = c < CLK ? cluster.map_shared_rank(part, c) + j * RTC_PART_LD : nullptr;
 #pragma unroll
-                for (int c = 0; c < RTC_MAX_CLK; ++c)
-                    if (c < CLK) r += pv[c];
+                for (int v = 0; v < VB; ++v) {
+                    const int e = lane + 32 * (v0 + v);
+                    pv[v][c] = (c < CLK && e < E) ? src[e] : 0.f;
+                }
             }
-            logit[v] = r;
+#pragma unroll
+            for (int v = 0; v < VB; ++v) {
+                float r = 0.f;
+#pragma unroll
+                for (int c = 0; c < RTC_MAX_CLK; ++c)
+                    if (c < CLK) r += pv[v][c];
+                logit[v0 + v] = r;
+            }
         }
         router_select<EV>(p, t, logit, spbuf + warp * ROUTER_MAXV * 32, lane);
     }
