@@ -136,19 +136,20 @@ __device__ __forceinline__ void acc_bf16x8(float (&acc)[8], const uint4 &w) {
 }
 
 // y[n] = sum_{j<k} slot[pos(n, j)] (slot order) + osh[n], one warp per row, each
-// lane two 8-column pieces at a time.  The slot rows are fetched eight slots at
-// a time before any of them is added, so 16 slot loads and the shared row are in
-// flight per lane; the adds then run in slot order (a missing slot adds +0).
+// lane four 8-column pieces at a time.  The slot rows are fetched eight slots at
+// a time before any of them is added, so 32 slot loads and the shared row are in
+// flight per lane (the phase is bound by load latency at one CTA of six warps per
+// SM); the adds then run in slot order (a missing slot adds +0).
 __device__ __forceinline__ void combine_rows(const GemmArgs &a, int gwarp, int nwarps, int lane) {
+    constexpr int U = 4;
     const int pieces = a.ncols_s / 8;
     for (int n = gwarp; n < a.N; n += nwarps) {
         const int my_pos = lane < a.k ? a.pos_of[(size_t)n * a.k + lane] : -1;
-        // Uniform trip count across the warp: the shuffles below need every lane.
-        for (int pbase = 0; pbase < pieces; pbase += 64) {
+        for (int pbase = 0; pbase < pieces; pbase += 32 * U) {
             const int p0 = pbase + lane;
-            float4 o[2][2];
+            float4 o[U][2];
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
+            for (int u = 0; u < U; ++u) {
                 const int pc = p0 + 32 * u;
                 if (pc < pieces) {
                     const float4 *op = reinterpret_cast<const float4 *>(a.osh + (size_t)n * a.ld_s + pc * 8);
@@ -156,19 +157,19 @@ __device__ __forceinline__ void combine_rows(const GemmArgs &a, int gwarp, int n
                     o[u][1] = __ldcg(op + 1);
                 }
             }
-            float sum[2][8];
+            float sum[U][8];
 #pragma unroll
-            for (int u = 0; u < 2; ++u)
+            for (int u = 0; u < U; ++u)
 #pragma unroll
                 for (int h = 0; h < 8; ++h) sum[u][h] = 0.f;
             for (int jb = 0; jb < a.k; jb += 8) {
-                uint4 w[8][2];
+                uint4 w[8][U];
 #pragma unroll
                 for (int jj = 0; jj < 8; ++jj) {
                     const int j = jb + jj;
                     const int p = __shfl_sync(0xffffffffu, my_pos, j & 31);
 #pragma unroll
-                    for (int u = 0; u < 2; ++u) {
+                    for (int u = 0; u < U; ++u) {
                         const int pc = p0 + 32 * u;
                         w[jj][u] = make_uint4(0u, 0u, 0u, 0u);
                         if (j < a.k && p >= 0 && pc < pieces)
@@ -179,10 +180,10 @@ __device__ __forceinline__ void combine_rows(const GemmArgs &a, int gwarp, int n
 #pragma unroll
                 for (int jj = 0; jj < 8; ++jj)
 #pragma unroll
-                    for (int u = 0; u < 2; ++u) acc_bf16x8(sum[u], w[jj][u]);
+                    for (int u = 0; u < U; ++u) acc_bf16x8(sum[u], w[jj][u]);
             }
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
+            for (int u = 0; u < U; ++u) {
                 const int pc = p0 + 32 * u;
                 if (pc < pieces) {
                     const float4 o0 = o[u][0], o1 = o[u][1];
