@@ -198,6 +198,87 @@ int moe_debug_never_signal(int on);
 int moe_profile_set_events(void *const *events, int n);
 unsigned long long moe_launch_count(void);
 
+/* ------------------------------------------------------------------------- *
+ * Expert parallelism over peer memory.
+ *
+ * "GLM-5.3-Flash Module 02" (expert placement and popularity) treats the
+ * placement of experts across devices as a serving variable: each token's
+ * hidden state is sent to the devices that hold its top-k experts and the
+ * expert outputs come back.  Here P ranks (one process per GPU, P <= 8) each
+ * hold E/P experts, rank q the experts [q*E/P, (q+1)*E/P), and their own batch
+ * of tokens.  The exchange is done by the kernels themselves: stores and
+ * atomics into the other ranks' memory over NVLink / NVSwitch, with bounded
+ * waits on counters, no collective-library call.
+ *
+ * Every rank owns a symmetric buffer of moe_ep_symmetric_bytes() bytes (the
+ * same P, N_cap, D, E, k on every rank), zero-filled once before the first
+ * call, and maps every other rank's buffer into its own address space
+ * (moe_ep_ipc_export / moe_ep_ipc_open).  peer_sym[q] is rank q's buffer as
+ * seen from the calling rank (peer_sym[rank] = its own); 256-byte aligned.
+ *
+ * moe_ep_forward computes, for the calling rank's N <= N_cap tokens, the same
+ * y as moe_forward would with all E experts on one device (bf16 only; the
+ * per-row arithmetic is that of moe_forward's 128-row-tile kernels, so y equals
+ * moe_forward's bit for bit whenever moe_forward takes those kernels, N > 256).
+ *   gate_up_loc [E/P, 2*d_moe, D] and down_loc [E/P, D, d_moe]: this rank's
+ *   experts; sh_*: the shared expert (replicated); topk_idx/topk_w [N, k] with
+ *   global expert ids (id E is the sentinel, skipped).
+ *   epoch: 1, 2, 3, ... the number of this call, equal on all ranks.
+ *   phases: a mask of MOE_EP_COUNT (publish this rank's expert histogram to all
+ *   ranks), MOE_EP_SEND (wait for all histograms, store token rows into the
+ *   owners' buffers), MOE_EP_EXPERTS (wait for this rank's rows, run its
+ *   experts and the shared expert, store weighted rows back into the sources'
+ *   buffers) and MOE_EP_COMBINE (wait for this rank's rows to come back, write
+ *   y).  A multi-GPU job passes MOE_EP_ALL on every rank.  Running the phases
+ *   one at a time over all ranks lets P ranks run on one device, since every
+ *   wait is then already satisfied.
+ *   workspace: moe_ep_workspace_bytes() bytes, 256-byte aligned, private to the
+ *   rank and kept between the phases of one epoch.
+ * Errors: MOE_ERR_ARG (phases, P, rank, epoch, pointers), MOE_ERR_SHAPE
+ * (E % P, E > 512, k, N > N_cap, D / d_moe / d_sh not multiples of 8),
+ * MOE_ERR_WORKSPACE; a wait that runs out (a rank that never arrives) is
+ * reported by moe_device_status as MOE_ERR_DEVICE_TIMEOUT.
+ */
+#define MOE_EP_COUNT 1
+#define MOE_EP_SEND 2
+#define MOE_EP_EXPERTS 4
+#define MOE_EP_COMBINE 8
+#define MOE_EP_ALL 15
+#define MOE_EP_MAX_RANKS 8
+#define MOE_EP_IPC_HANDLE_BYTES 72 /* CUDA IPC handle (64) + offset in its allocation (8) */
+
+size_t moe_ep_symmetric_bytes(int P, int N_cap, int D, int E, int k);
+size_t moe_ep_workspace_bytes(int P, int N_cap, int D, int E, int d_moe, int d_sh, int k);
+int moe_ep_forward(int phases, int P, int rank, unsigned epoch, void *const *peer_sym, int N_cap,
+                   const void *x, const void *gate_up_loc, const void *down_loc,
+                   const void *sh_gate, const void *sh_up, const void *sh_down,
+                   const int32_t *topk_idx, const float *topk_w, int N, int D, int E, int d_moe,
+                   int d_sh, int k, void *y, void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * moe_ep_plan_host — the layout the send phase derives, computed on the host
+ * (no device needed): from the P x E histogram counts[r][e] (pairs of rank r
+ * routed to expert e), for sender `rank`: dest_base[e] = the row, in expert
+ * e's owner's receive buffer, of this rank's first pair routed to e, minus
+ * that pair's position in this rank's expert-sorted order; for `rank` as a
+ * receiver: rcounts[E/P] rows per local expert, rtile_off[E/P + 1] the prefix
+ * of 128-row tiles, *rows_in rows received, *pairs_out pairs sent.
+ */
+int moe_ep_plan_host(int P, int rank, int E, const int32_t *counts, int32_t *dest_base,
+                     int32_t *rcounts, int32_t *rtile_off, int32_t *rows_in, int32_t *pairs_out);
+
+/*
+ * Mapping another rank's symmetric buffer (CUDA IPC).  moe_ep_ipc_export writes
+ * MOE_EP_IPC_HANDLE_BYTES bytes naming dev_ptr (any address inside a device
+ * allocation of this process); another process's moe_ep_ipc_open maps it and
+ * returns the same address in its own space; moe_ep_ipc_close unmaps a pointer
+ * returned by moe_ep_ipc_open.  MOE_ERR_CUDA if the driver refuses (e.g. the
+ * same process, or no peer access).
+ */
+int moe_ep_ipc_export(const void *dev_ptr, void *handle);
+int moe_ep_ipc_open(const void *handle, void **dev_ptr);
+int moe_ep_ipc_close(void *dev_ptr);
+
 #ifdef __cplusplus
 }
 #endif

@@ -21,7 +21,10 @@ __all__ = ["MoEError", "moe_router", "moe_forward", "moe_forward_workspace", "mo
            "moe_device_status", "moe_status_string", "moe_debug_set_wait_limit_ns",
            "moe_debug_never_signal", "moe_profile_set_events", "moe_launch_count",
            "moe_forward_noalloc", "library_path", "load_library", "MOE_F32", "MOE_BF16",
-           "EXPORTED_SYMBOLS"]
+           "EXPORTED_SYMBOLS", "moe_ep_symmetric_bytes", "moe_ep_workspace_bytes",
+           "moe_ep_forward", "moe_ep_plan_host", "moe_ep_ipc_export", "moe_ep_ipc_open",
+           "moe_ep_ipc_close", "ExpertParallelGroup", "MOE_EP_COUNT", "MOE_EP_SEND",
+           "MOE_EP_EXPERTS", "MOE_EP_COMBINE", "MOE_EP_ALL"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libmoe.so")
@@ -30,11 +33,17 @@ _lib = None
 
 MOE_F32, MOE_BF16 = 0, 1
 MOE_OK = 0
+MOE_EP_COUNT, MOE_EP_SEND, MOE_EP_EXPERTS, MOE_EP_COMBINE = 1, 2, 4, 8
+MOE_EP_ALL = 15
+MOE_EP_PHASES = (MOE_EP_COUNT, MOE_EP_SEND, MOE_EP_EXPERTS, MOE_EP_COMBINE)
+MOE_EP_IPC_HANDLE_BYTES = 72
 
 EXPORTED_SYMBOLS = ("moe_router", "moe_forward_workspace", "moe_forward", "moe_device_status",
                     "moe_status_string", "moe_version", "moe_debug_set_wait_limit_ns",
                     "moe_debug_never_signal", "moe_profile_set_events", "moe_launch_count",
-                    "moe_forward_noalloc", "moe_forward_clamped")
+                    "moe_forward_noalloc", "moe_forward_clamped", "moe_ep_symmetric_bytes",
+                    "moe_ep_workspace_bytes", "moe_ep_forward", "moe_ep_plan_host",
+                    "moe_ep_ipc_export", "moe_ep_ipc_open", "moe_ep_ipc_close")
 
 
 class MoEError(RuntimeError):
@@ -84,6 +93,22 @@ def load_library():
         lib.moe_forward_clamped.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, F, P,
                                             P, ctypes.c_size_t, P]
         lib.moe_forward_clamped.restype = I
+        S = ctypes.c_size_t
+        lib.moe_ep_symmetric_bytes.argtypes = [I, I, I, I, I]
+        lib.moe_ep_symmetric_bytes.restype = S
+        lib.moe_ep_workspace_bytes.argtypes = [I, I, I, I, I, I, I]
+        lib.moe_ep_workspace_bytes.restype = S
+        lib.moe_ep_forward.argtypes = [I, I, I, ctypes.c_uint, ctypes.POINTER(ctypes.c_void_p), I,
+                                       P, P, P, P, P, P, P, P, I, I, I, I, I, I, P, P, S, P]
+        lib.moe_ep_forward.restype = I
+        lib.moe_ep_plan_host.argtypes = [I, I, I, P, P, P, P, P, P]
+        lib.moe_ep_plan_host.restype = I
+        lib.moe_ep_ipc_export.argtypes = [P, P]
+        lib.moe_ep_ipc_export.restype = I
+        lib.moe_ep_ipc_open.argtypes = [P, ctypes.POINTER(ctypes.c_void_p)]
+        lib.moe_ep_ipc_open.restype = I
+        lib.moe_ep_ipc_close.argtypes = [P]
+        lib.moe_ep_ipc_close.restype = I
         _lib = lib
         return lib
 
@@ -242,3 +267,124 @@ def moe_profile_set_events(events) -> None:
 
 def moe_launch_count() -> int:
     return int(load_library().moe_launch_count())
+
+
+# ----------------------------------------------------------------------------- experts
+# spread over ranks (peer memory; see include/moe.h, "Expert parallelism")
+
+def moe_ep_symmetric_bytes(P: int, N_cap: int, D: int, E: int, k: int) -> int:
+    return int(load_library().moe_ep_symmetric_bytes(P, N_cap, D, E, k))
+
+
+def moe_ep_workspace_bytes(P: int, N_cap: int, D: int, E: int, d_moe: int, d_sh: int,
+                           k: int) -> int:
+    return int(load_library().moe_ep_workspace_bytes(P, N_cap, D, E, d_moe, d_sh, k))
+
+
+def moe_ep_forward(phases: int, P: int, rank: int, epoch: int, peer_sym, N_cap: int, x, gate_up_loc,
+                   down_loc, sh_gate, sh_up, sh_down, topk_idx, topk_w, E: int, y, workspace,
+                   stream=None):
+    """One rank's part of an expert-parallel forward.  peer_sym: the P symmetric buffers'
+    device addresses as seen from this rank; gate_up_loc / down_loc: this rank's E/P
+    experts; topk_idx holds global expert ids.  y [N, D] must be preallocated."""
+    lib = load_library()
+    N, D = x.shape
+    E_loc, two_d, _ = gate_up_loc.shape
+    k = topk_idx.shape[1]
+    arr = (ctypes.c_void_p * P)(*[int(a) for a in peer_sym])
+    dp = lambda t, name: _dev(t, name) if t.numel() else 0
+    rc = lib.moe_ep_forward(phases, P, rank, epoch, arr, N_cap, dp(x, "x"),
+                            _dev(gate_up_loc, "gate_up_loc"), _dev(down_loc, "down_loc"),
+                            _dev(sh_gate, "sh_gate"), _dev(sh_up, "sh_up"), _dev(sh_down, "sh_down"),
+                            dp(topk_idx, "topk_idx"), dp(topk_w, "topk_w"), N, D, E, two_d // 2,
+                            sh_gate.shape[0], k, dp(y, "y"), _dev(workspace, "workspace"),
+                            workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc, "moe_ep_forward")
+    return y
+
+
+def moe_ep_plan_host(P: int, rank: int, counts):
+    """Host mirror of the send-phase layout from the P x E histogram (numpy int32)."""
+    import numpy as np
+    counts = np.ascontiguousarray(counts, dtype=np.int32)
+    Pc, E = counts.shape
+    if Pc != P:
+        raise ValueError("counts must be [P, E]")
+    E_loc = E // P if P else 0
+    dest = np.zeros(E, np.int32)
+    rc_ = np.zeros(max(E_loc, 1), np.int32)
+    rto = np.zeros(E_loc + 1, np.int32)
+    rows_in = ctypes.c_int32(0)
+    pairs_out = ctypes.c_int32(0)
+    ptr = lambda a: a.ctypes.data_as(ctypes.c_void_p)
+    rc = load_library().moe_ep_plan_host(P, rank, E, ptr(counts), ptr(dest), ptr(rc_), ptr(rto),
+                                         ctypes.byref(rows_in), ctypes.byref(pairs_out))
+    _check(rc, "moe_ep_plan_host")
+    return {"dest_base": dest, "rcounts": rc_[:E_loc], "rtile_off": rto,
+            "rows_in": int(rows_in.value), "pairs_out": int(pairs_out.value)}
+
+
+def moe_ep_ipc_export(t: torch.Tensor) -> bytes:
+    buf = ctypes.create_string_buffer(MOE_EP_IPC_HANDLE_BYTES)
+    _check(load_library().moe_ep_ipc_export(_dev(t, "buffer"), buf), "moe_ep_ipc_export")
+    return buf.raw
+
+
+def moe_ep_ipc_open(handle: bytes) -> int:
+    out = ctypes.c_void_p()
+    buf = ctypes.create_string_buffer(bytes(handle), MOE_EP_IPC_HANDLE_BYTES)
+    _check(load_library().moe_ep_ipc_open(buf, ctypes.byref(out)), "moe_ep_ipc_open")
+    return int(out.value)
+
+
+def moe_ep_ipc_close(ptr: int) -> None:
+    _check(load_library().moe_ep_ipc_close(ctypes.c_void_p(ptr)), "moe_ep_ipc_close")
+
+
+class ExpertParallelGroup:
+    """Expert-parallel layer state of one rank in a torch.distributed job (one process per
+    GPU): allocates this rank's symmetric buffer and workspace, exchanges CUDA IPC handles
+    with the other ranks (all_gather_object over the default group) and maps their
+    buffers.  forward() runs all four phases for the next epoch."""
+
+    def __init__(self, N_cap: int, D: int, E: int, k: int, d_moe: int, d_sh: int, device=None,
+                 group=None):
+        import torch.distributed as dist
+        self.P = dist.get_world_size(group)
+        self.rank = dist.get_rank(group)
+        self.N_cap, self.E = N_cap, E
+        dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+        sym_bytes = moe_ep_symmetric_bytes(self.P, N_cap, D, E, k)
+        ws_bytes = moe_ep_workspace_bytes(self.P, N_cap, D, E, d_moe, d_sh, k)
+        if not sym_bytes or not ws_bytes:
+            raise ValueError("unsupported expert-parallel shape")
+        self.sym = torch.zeros(sym_bytes, dtype=torch.uint8, device=dev)
+        self.workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+        torch.cuda.synchronize(dev)
+        handles = [None] * self.P
+        dist.all_gather_object(handles, moe_ep_ipc_export(self.sym), group=group)
+        self._opened = []
+        self.peer_sym = []
+        for q, h in enumerate(handles):
+            if q == self.rank:
+                self.peer_sym.append(self.sym.data_ptr())
+            else:
+                ptr = moe_ep_ipc_open(h)
+                self._opened.append(ptr)
+                self.peer_sym.append(ptr)
+        dist.barrier(group=group)
+        self.epoch = 0
+
+    def forward(self, x, gate_up_loc, down_loc, sh_gate, sh_up, sh_down, topk_idx, topk_w,
+                y=None, stream=None):
+        if y is None:
+            y = torch.empty_like(x)
+        self.epoch += 1
+        return moe_ep_forward(MOE_EP_ALL, self.P, self.rank, self.epoch, self.peer_sym, self.N_cap,
+                              x, gate_up_loc, down_loc, sh_gate, sh_up, sh_down, topk_idx, topk_w,
+                              self.E, y, self.workspace, stream)
+
+    def close(self):
+        for ptr in self._opened:
+            moe_ep_ipc_close(ptr)
+        self._opened = []

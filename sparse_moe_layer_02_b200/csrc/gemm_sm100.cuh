@@ -49,6 +49,27 @@ constexpr int GEMM_SMEM_BYTES =
 
 enum GemmKind { GEMM_GATE_UP = 0, GEMM_DOWN = 1 };
 
+constexpr int EP_MAX_RANKS = 8; // ranks of an expert-parallel group
+
+__device__ __forceinline__ uint32_t ld_acquire_sys_u32(const uint32_t *p) {
+    uint32_t v;
+    asm volatile("ld.acquire.sys.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Adds 1 to ctr[key] for every lane of the calling (converged) warp with key in
+// [0, nkeys), one atomic per distinct key, after the earlier stores of every lane
+// of the warp are visible system-wide (they may be in another GPU's memory): each
+// lane fences its own stores, the warp barrier orders all lanes before the
+// leaders' atomics.
+__device__ __forceinline__ void warp_count_rows(uint32_t *const *ctr, int key, int nkeys) {
+    __threadfence_system();
+    __syncwarp();
+    const bool ok = key >= 0 && key < nkeys;
+    const uint32_t same = __match_any_sync(0xffffffffu, ok ? key : -1);
+    if (ok && (__ffs(same) - 1) == (int)(threadIdx.x & 31)) atomicAdd(ctr[key], (uint32_t)__popc(same));
+}
+
 struct GemmArgs {
     const int32_t *tile_off; // [E+1]
     int32_t *meta;           // [0] routed tiles done (down), [2] routed m-tiles
@@ -70,6 +91,14 @@ struct GemmArgs {
     uint64_t wait_limit_ns;
     int never_signal;
     float gate_max, up_max; // gate_up: SwiGLU limits (+infinity = plain SwiGLU)
+    // Expert parallelism (all null / 0 for a single-device layer).  The routed
+    // rows are other ranks' tokens received into this rank's buffer.
+    const uint32_t *ep_wait_ctr;    // gate_up: rows arrived (this epoch) ...
+    const int32_t *ep_wait_target;  // ... must reach *ep_wait_target before any load
+    const int4 *ep_meta;            // down: per routed row {source rank or -1, pair id, w bits, 0}
+    int ep_P;                       // down: ranks; > 0 selects the expert-parallel epilogue
+    __nv_bfloat16 *ep_out[EP_MAX_RANKS]; // down: every rank's slot buffer (rows by pair id)
+    uint32_t *ep_ret[EP_MAX_RANKS];      // down: every rank's returned-rows counter (this epoch)
 };
 
 struct TileCoord {
@@ -252,9 +281,27 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
-    const int routed_tiles = a.meta[2] * a.nb_r;
-    const int total_tiles = routed_tiles + a.mt_s * a.nb_s;
     const uint64_t limit = a.wait_limit_ns;
+    if (a.ep_wait_ctr) {
+        // Expert parallelism: other ranks write the routed rows; start once all of
+        // them have arrived (bounded wait), and make the rows visible to TMA.
+        if (threadIdx.x == 0) {
+            const uint32_t target = (uint32_t)*a.ep_wait_target;
+            const uint64_t t0 = globaltimer_ns();
+            while (ld_acquire_sys_u32(a.ep_wait_ctr) < target) {
+                if (globaltimer_ns() - t0 > limit) {
+                    record_error(DEV_TIMEOUT, 104);
+                    *abort_flag = 1;
+                    break;
+                }
+                __nanosleep(128);
+            }
+            fence_proxy_async_global();
+        }
+        __syncthreads();
+    }
+    const int routed_tiles = a.meta[2] * a.nb_r;
+    const int total_tiles = *abort_flag ? 0 : routed_tiles + a.mt_s * a.nb_s;
 
     if (warp == 0) {
         // ------------------------------ TMA producer ------------------------------
@@ -384,21 +431,34 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 }
             } else if (!c.shared) {
                 const int grow = c.a_row + row;
-                const float wr = a.w_perm[grow];
-                __nv_bfloat16 *row_ptr = a.out_r + (size_t)grow * a.ld_r;
+                float wr;
+                __nv_bfloat16 *row_ptr;
+                int src = 0;
+                if (a.ep_P > 0) {
+                    // the row goes back to its token's rank, at the token's pair id;
+                    // padding rows carry source -1 and are not stored
+                    const int4 m = a.ep_meta[grow];
+                    src = (m.x >= 0 && m.x < a.ep_P) ? m.x : -1;
+                    wr = __int_as_float(m.z);
+                    row_ptr = src >= 0 ? a.ep_out[src] + (size_t)m.y * a.ld_r : nullptr;
+                } else {
+                    wr = a.w_perm[grow];
+                    row_ptr = a.out_r + (size_t)grow * a.ld_r;
+                }
 #pragma unroll 1
                 for (int ch = 0; ch < 8; ++ch) {
                     uint32_t v[32];
                     tmem_ld_32x32b_x32(tbase + ch * 32, v);
                     tmem_ld_wait();
                     const int col = c.nb * GEMM_BN + ch * 32;
-                    if (col < a.ncols_r) {
+                    if (row_ptr && col < a.ncols_r) {
                         float o[32];
 #pragma unroll
                         for (int i = 0; i < 32; ++i) o[i] = wr * __uint_as_float(v[i]);
                         store_row_chunk_bf16(row_ptr, col, a.ncols_r, o);
                     }
                 }
+                if (a.ep_P > 0) warp_count_rows(a.ep_ret, src, a.ep_P);
             } else {
                 // shared expert: fp32 output rows, combined after every tile is done
                 const int n = c.a_row + row;
@@ -440,7 +500,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         tmem_dealloc(tmem_base, GEMM_TMEM_COLS);
     }
 
-    if (KIND == GEMM_DOWN) {
+    if (KIND == GEMM_DOWN && a.ep_P == 0) {
         // ---- combine phase: every tile of the launch must be stored first ----------
         if (threadIdx.x == 0 && !*abort_flag) {
             const int target = total_tiles + (a.never_signal ? 1 : 0);

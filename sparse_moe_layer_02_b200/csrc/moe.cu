@@ -4,11 +4,13 @@
 #include <cudaTypedefs.h>
 
 #include <atomic>
+#include <cstring>
 #include <mutex>
 
 #include "moe.h"
 #include "common.cuh"
 #include "dispatch.cuh"
+#include "ep.cuh"
 #include "gemm_decode_sm100.cuh"
 #include "gemm_sm100.cuh"
 #include "router.cuh"
@@ -738,6 +740,364 @@ int moe_device_status(void *stream) {
     if (s.error == DEV_TIMEOUT) return MOE_ERR_DEVICE_TIMEOUT;
     if (s.error == DEV_BAD_INDEX) return MOE_ERR_BAD_INDEX;
     return MOE_OK;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Expert parallelism (peer memory): workspace, launch sequence, IPC mapping.
+// ---------------------------------------------------------------------------
+namespace moe {
+namespace {
+
+struct EpWs {
+    size_t chunk_hist, counts, dense_off, dmeta, pos_of, perm_tok, w_perm;
+    size_t dest_base, rcounts, rtile_off, rmeta, pair_pos;
+    size_t h_perm, h_sh, osh, total;
+    int nchunks;
+};
+
+bool plan_ep(int P, int N_cap, int D, int E, int d, int d_sh, int k, EpSym &S, EpWs &W) {
+    if (!ep_sym_layout(P, N_cap, D, E, k, S)) return false;
+    if (d <= 0 || d_sh <= 0) return false;
+    const size_t nk = (size_t)N_cap * k;
+    if (nk > (size_t)INT32_MAX / 4) return false;
+    W.nchunks = (int)((nk + DISPATCH_CHUNK - 1) / DISPATCH_CHUNK);
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = off;
+        off = round_up(off + bytes, 256);
+        return at;
+    };
+    const int E_loc = E / P;
+    W.chunk_hist = take((size_t)std::max(W.nchunks, 1) * E * 4);
+    W.counts = take((size_t)E * 4);
+    W.dense_off = take((size_t)(E + 1) * 4);
+    W.dmeta = take(16 * 4);
+    W.pos_of = take(std::max<size_t>(nk, 1) * 4);
+    W.perm_tok = take(std::max<size_t>(nk, 1) * 4);
+    W.w_perm = take(std::max<size_t>(nk, 1) * 4);
+    W.dest_base = take((size_t)E * 4);
+    W.rcounts = take((size_t)E_loc * 4);
+    W.rtile_off = take((size_t)(E_loc + 1) * 4);
+    W.rmeta = take(16 * 4);
+    W.pair_pos = take(std::max<size_t>(nk, 1) * 4);
+    W.h_perm = take((size_t)S.rows_cap * d * 2);
+    W.h_sh = take(std::max<size_t>((size_t)N_cap * d_sh * 2, 16));
+    W.osh = take(std::max<size_t>((size_t)N_cap * D * 4, 16));
+    W.total = off;
+    return true;
+}
+
+int ep_forward_impl(int phases, int P, int rank, uint32_t epoch, void *const *peer_sym, int N_cap,
+                    const void *x, const void *gate_up_loc, const void *down_loc,
+                    const void *sh_gate, const void *sh_up, const void *sh_down,
+                    const int32_t *topk_idx, const float *topk_w, int N, int D, int E, int d_moe,
+                    int d_sh, int k, void *y, void *workspace, size_t ws_bytes, void *stream) {
+    if (phases <= 0 || phases > MOE_EP_ALL) return MOE_ERR_ARG;
+    if (P < 1 || P > EP_MAX_RANKS || rank < 0 || rank >= P || epoch == 0) return MOE_ERR_ARG;
+    if (E <= 0 || E > DISPATCH_MAXE || E % P || k <= 0 || k > 32 || k > E) return MOE_ERR_SHAPE;
+    if (N < 0 || N > N_cap || D <= 0 || d_moe <= 0 || d_sh <= 0) return MOE_ERR_SHAPE;
+    if (D % 8 || d_moe % 8 || d_sh % 8) return MOE_ERR_SHAPE;
+    EpSym S;
+    EpWs W;
+    if (!plan_ep(P, N_cap, D, E, d_moe, d_sh, k, S, W)) return MOE_ERR_SHAPE;
+    if (!peer_sym) return MOE_ERR_ARG;
+    for (int q = 0; q < P; ++q)
+        if (!peer_sym[q] || (reinterpret_cast<uintptr_t>(peer_sym[q]) & 255u)) return MOE_ERR_ARG;
+    const void *ptrs[] = {gate_up_loc, down_loc, sh_gate, sh_up, sh_down};
+    for (const void *q : ptrs)
+        if (!q || !aligned16(q)) return MOE_ERR_ARG;
+    if (N > 0) {
+        const void *io[] = {x, topk_idx, topk_w, y};
+        for (const void *q : io)
+            if (!q || !aligned16(q)) return MOE_ERR_ARG;
+    }
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return MOE_ERR_WORKSPACE;
+    if (ws_bytes < W.total) return MOE_ERR_WORKSPACE;
+    int rc;
+    DeviceInfo *dev = nullptr;
+    if ((rc = current_device_info(&dev)) != MOE_OK) return rc;
+    if (dev->major != 10) return MOE_ERR_NO_DEVICE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    Profiler prof(st);
+    const int E_loc = E / P;
+    const int par = epoch & 1;
+
+    EpParams ep = {};
+    ep.P = P;
+    ep.rank = rank;
+    ep.E = E;
+    ep.E_loc = E_loc;
+    ep.k = k;
+    ep.N = N;
+    ep.D = D;
+    ep.epoch = epoch;
+    for (int q = 0; q < P; ++q) ep.sym[q] = static_cast<uint8_t *>(peer_sym[q]);
+    ep.S = S;
+    ep.x = static_cast<const uint8_t *>(x);
+    ep.topk_idx = topk_idx;
+    ep.topk_w = topk_w;
+    ep.counts = reinterpret_cast<int32_t *>(ws + W.counts);
+    ep.dense_off = reinterpret_cast<int32_t *>(ws + W.dense_off);
+    ep.pos_of = reinterpret_cast<int32_t *>(ws + W.pos_of);
+    ep.dest_base = reinterpret_cast<int32_t *>(ws + W.dest_base);
+    ep.rcounts = reinterpret_cast<int32_t *>(ws + W.rcounts);
+    ep.rtile_off = reinterpret_cast<int32_t *>(ws + W.rtile_off);
+    ep.rmeta = reinterpret_cast<int32_t *>(ws + W.rmeta);
+    ep.pair_pos = reinterpret_cast<int32_t *>(ws + W.pair_pos);
+    ep.down_nb = (D + GEMM_BN - 1) / GEMM_BN;
+    ep.wait_limit_ns = g_wait_limit_ns;
+
+    if (phases & MOE_EP_COUNT) {
+        // dense dispatch of this rank's pairs (one-row tiles: positions are
+        // expert-sorted with no padding)
+        DispatchParams dp;
+        dp.topk_idx = topk_idx;
+        dp.topk_w = topk_w;
+        dp.N = N;
+        dp.k = k;
+        dp.E = E;
+        dp.nchunks = W.nchunks;
+        dp.tile_rows = 1;
+        dp.chunk_hist = reinterpret_cast<int32_t *>(ws + W.chunk_hist);
+        dp.counts = reinterpret_cast<int32_t *>(ws + W.counts);
+        dp.tile_off = reinterpret_cast<int32_t *>(ws + W.dense_off);
+        dp.meta = reinterpret_cast<int32_t *>(ws + W.dmeta);
+        dp.pos_of = reinterpret_cast<int32_t *>(ws + W.pos_of);
+        dp.perm_tok = reinterpret_cast<int32_t *>(ws + W.perm_tok);
+        dp.w_perm = reinterpret_cast<float *>(ws + W.w_perm);
+        if ((size_t)N * k <= DISPATCH_SMALL_IDS) {
+            dispatch_small_kernel<<<1, DISPATCH_SMALL_THREADS, 0, st>>>(dp);
+            if ((rc = launched(prof)) != MOE_OK) return rc;
+        } else {
+            dp.nchunks = (int)(((size_t)N * k + DISPATCH_CHUNK - 1) / DISPATCH_CHUNK);
+            dispatch_count_kernel<<<dp.nchunks, DISPATCH_THREADS, 0, st>>>(dp);
+            if ((rc = launched(prof)) != MOE_OK) return rc;
+            dispatch_scan_kernel<<<1, DISPATCH_MAXE, 0, st>>>(dp);
+            if ((rc = launched(prof)) != MOE_OK) return rc;
+            dispatch_scatter_kernel<<<dp.nchunks, DISPATCH_THREADS, 0, st>>>(dp);
+            if ((rc = launched(prof)) != MOE_OK) return rc;
+        }
+        ep_publish_kernel<<<1, 512, 0, st>>>(ep);
+        if ((rc = launched(prof)) != MOE_OK) return rc;
+    }
+    if (phases & MOE_EP_SEND) {
+        ep_layout_kernel<<<1, 512, 0, st>>>(ep);
+        if ((rc = launched(prof)) != MOE_OK) return rc;
+        if (N > 0) {
+            const int items = N * ((D * 2 / 16 + EP_PIECE_VEC - 1) / EP_PIECE_VEC);
+            const int grid = std::min((items + 7) / 8, dev->sms * 16);
+            ep_send_kernel<<<grid, 256, 0, st>>>(ep);
+            if ((rc = launched(prof)) != MOE_OK) return rc;
+        }
+    }
+    uint8_t *own = ep.sym[rank];
+    if (phases & MOE_EP_EXPERTS) {
+        if ((rc = ensure_gemm_attrs(dev)) != MOE_OK) return rc;
+        const void *recv_x = own + S.recv_x;
+        __nv_bfloat16 *h_perm = reinterpret_cast<__nv_bfloat16 *>(ws + W.h_perm);
+        __nv_bfloat16 *h_sh = reinterpret_cast<__nv_bfloat16 *>(ws + W.h_sh);
+        const uint64_t nrows = std::max(N, 1); // maps need a row; no tile reads past N
+        CUtensorMap mx_perm, mgu, mx, msg, msu, mh_perm, mdn, mh_sh, msd;
+        const bool ok = make_map(&mx_perm, recv_x, D, S.rows_cap, D, 128) &&
+                        make_map(&mgu, gate_up_loc, D, (uint64_t)E_loc * 2 * d_moe, D, 128) &&
+                        make_map(&mx, N > 0 ? x : recv_x, D, nrows, D, 128) &&
+                        make_map(&msg, sh_gate, D, d_sh, D, 128) &&
+                        make_map(&msu, sh_up, D, d_sh, D, 128) &&
+                        make_map(&mh_perm, h_perm, d_moe, S.rows_cap, d_moe, 128) &&
+                        make_map(&mdn, down_loc, d_moe, (uint64_t)E_loc * D, d_moe, GEMM_BN) &&
+                        make_map(&mh_sh, h_sh, d_sh, nrows, d_sh, 128) &&
+                        make_map(&msd, sh_down, d_sh, D, d_sh, GEMM_BN);
+        if (!ok) return MOE_ERR_CUDA;
+        const int mt_s = (N + GEMM_BM - 1) / GEMM_BM;
+        const int mt_r_max = S.rows_cap / GEMM_BM;
+        GemmArgs g = {};
+        g.tile_off = ep.rtile_off;
+        g.meta = ep.rmeta;
+        g.E = E_loc;
+        g.N = N;
+        g.k = k;
+        g.mt_s = mt_s;
+        g.wait_limit_ns = g_wait_limit_ns;
+        g.gate_max = INFINITY;
+        g.up_max = INFINITY;
+        g.nb_r = (d_moe + 127) / 128;
+        g.nb_s = (d_sh + 127) / 128;
+        g.kb_r = g.kb_s = (D + GEMM_BK - 1) / GEMM_BK;
+        g.b_rows_per_e = 2 * d_moe;
+        g.up_off = d_moe;
+        g.out_r = h_perm;
+        g.ld_r = g.ncols_r = d_moe;
+        g.out_s = h_sh;
+        g.ld_s = g.ncols_s = d_sh;
+        g.ep_wait_ctr = reinterpret_cast<const uint32_t *>(own + S.ctr) + par;
+        g.ep_wait_target = ep.rmeta + 3;
+        int max_tiles = mt_r_max * g.nb_r + mt_s * g.nb_s;
+        rc = launch_gemm<GEMM_GATE_UP>(mx_perm, mgu, mx, msg, msu, g, std::min(dev->sms, max_tiles),
+                                       false, st);
+        prof.mark();
+        if (rc != MOE_OK) return rc;
+        g.ep_wait_ctr = nullptr;
+        g.ep_wait_target = nullptr;
+        g.nb_r = g.nb_s = (D + GEMM_BN - 1) / GEMM_BN;
+        g.kb_r = (d_moe + GEMM_BK - 1) / GEMM_BK;
+        g.kb_s = (d_sh + GEMM_BK - 1) / GEMM_BK;
+        g.b_rows_per_e = D;
+        g.up_off = 0;
+        g.out_r = nullptr;
+        g.ld_r = g.ncols_r = D;
+        g.out_s = static_cast<__nv_bfloat16 *>(y);
+        g.ld_s = g.ncols_s = D;
+        g.osh = reinterpret_cast<float *>(ws + W.osh);
+        g.ep_P = P;
+        g.ep_meta = reinterpret_cast<const int4 *>(own + S.recv_meta);
+        for (int q = 0; q < P; ++q) {
+            g.ep_out[q] = reinterpret_cast<__nv_bfloat16 *>(ep.sym[q] + S.slot);
+            g.ep_ret[q] = reinterpret_cast<uint32_t *>(ep.sym[q] + S.ctr) + 2 + par;
+        }
+        max_tiles = mt_r_max * g.nb_r + mt_s * g.nb_s;
+        rc = launch_gemm<GEMM_DOWN>(mh_perm, mdn, mh_sh, msd, msd, g, std::min(dev->sms, max_tiles),
+                                    true, st);
+        prof.mark();
+        if (rc != MOE_OK) return rc;
+    }
+    if ((phases & MOE_EP_COMBINE) && N > 0) {
+        GemmArgs g = {};
+        g.N = N;
+        g.k = k;
+        g.ncols_s = g.ld_s = D;
+        g.ld_r = D;
+        g.out_s = static_cast<__nv_bfloat16 *>(y);
+        g.osh = reinterpret_cast<float *>(ws + W.osh);
+        g.pos_of = ep.pair_pos;
+        g.slot = reinterpret_cast<const __nv_bfloat16 *>(own + S.slot);
+        const int grid = std::min((N + 7) / 8, dev->sms * 4);
+        ep_combine_kernel<<<grid, 256, 0, st>>>(ep, g);
+        if ((rc = launched(prof)) != MOE_OK) return rc;
+    }
+    return MOE_OK;
+}
+
+// Host mirror of the layout the send phase derives on the device (see
+// ep_layout_kernel), for checks of the exchange logic without a GPU.
+int ep_plan_host(int P, int rank, int E, const int32_t *counts, int32_t *dest_base,
+                 int32_t *rcounts, int32_t *rtile_off, int32_t *rows_in, int32_t *pairs_out) {
+    if (P < 1 || P > EP_MAX_RANKS || rank < 0 || rank >= P || E <= 0 || E % P) return MOE_ERR_SHAPE;
+    if (!counts || !dest_base || !rcounts || !rtile_off || !rows_in || !pairs_out) return MOE_ERR_ARG;
+    const int E_loc = E / P;
+    int dense = 0, rin = 0, pout = 0;
+    for (int e = 0; e < E; ++e) {
+        const int q = e / E_loc, first = q * E_loc;
+        int tprefix = 0;
+        for (int e2 = first; e2 < e; ++e2) {
+            int R2 = 0;
+            for (int r = 0; r < P; ++r) R2 += counts[(size_t)r * E + e2];
+            tprefix += (R2 + EP_TILE - 1) / EP_TILE;
+        }
+        int R = 0, pre = 0;
+        for (int r = 0; r < P; ++r) {
+            R += counts[(size_t)r * E + e];
+            if (r < rank) pre += counts[(size_t)r * E + e];
+        }
+        dest_base[e] = tprefix * EP_TILE + pre - dense;
+        dense += counts[(size_t)rank * E + e];
+        pout += counts[(size_t)rank * E + e];
+        if (q == rank) {
+            rcounts[e - first] = R;
+            rtile_off[e - first] = tprefix;
+            rin += R;
+            if (e - first == E_loc - 1) rtile_off[E_loc] = tprefix + (R + EP_TILE - 1) / EP_TILE;
+        }
+    }
+    *rows_in = rin;
+    *pairs_out = pout;
+    return MOE_OK;
+}
+
+using PFN_getAddressRange = CUresult (*)(CUdeviceptr *, size_t *, CUdeviceptr);
+
+PFN_getAddressRange address_range_fn() {
+    static PFN_getAddressRange fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_getAddressRange>(p);
+    });
+    return fn;
+}
+
+}  // namespace
+}  // namespace moe
+
+extern "C" {
+
+size_t moe_ep_symmetric_bytes(int P, int N_cap, int D, int E, int k) {
+    moe::EpSym S;
+    return moe::ep_sym_layout(P, N_cap, D, E, k, S) ? S.total : 0;
+}
+
+size_t moe_ep_workspace_bytes(int P, int N_cap, int D, int E, int d_moe, int d_sh, int k) {
+    moe::EpSym S;
+    moe::EpWs W;
+    return moe::plan_ep(P, N_cap, D, E, d_moe, d_sh, k, S, W) ? W.total : 0;
+}
+
+int moe_ep_forward(int phases, int P, int rank, unsigned epoch, void *const *peer_sym, int N_cap,
+                   const void *x, const void *gate_up_loc, const void *down_loc,
+                   const void *sh_gate, const void *sh_up, const void *sh_down,
+                   const int32_t *topk_idx, const float *topk_w, int N, int D, int E, int d_moe,
+                   int d_sh, int k, void *y, void *workspace, size_t ws_bytes, void *stream) {
+    return moe::ep_forward_impl(phases, P, rank, epoch, peer_sym, N_cap, x, gate_up_loc, down_loc,
+                                sh_gate, sh_up, sh_down, topk_idx, topk_w, N, D, E, d_moe, d_sh, k,
+                                y, workspace, ws_bytes, stream);
+}
+
+int moe_ep_plan_host(int P, int rank, int E, const int32_t *counts, int32_t *dest_base,
+                     int32_t *rcounts, int32_t *rtile_off, int32_t *rows_in, int32_t *pairs_out) {
+    return moe::ep_plan_host(P, rank, E, counts, dest_base, rcounts, rtile_off, rows_in, pairs_out);
+}
+
+int moe_ep_ipc_export(const void *dev_ptr, void *handle) {
+    if (!dev_ptr || !handle) return MOE_ERR_ARG;
+    auto range = moe::address_range_fn();
+    if (!range) return MOE_ERR_CUDA;
+    CUdeviceptr base = 0;
+    size_t size = 0;
+    if (range(&base, &size, reinterpret_cast<CUdeviceptr>(dev_ptr)) != CUDA_SUCCESS) return MOE_ERR_CUDA;
+    cudaIpcMemHandle_t h;
+    if (cudaIpcGetMemHandle(&h, reinterpret_cast<void *>(base)) != cudaSuccess) return MOE_ERR_CUDA;
+    const uint64_t offset = reinterpret_cast<CUdeviceptr>(dev_ptr) - base;
+    std::memcpy(handle, &h, sizeof(h));
+    std::memcpy(static_cast<uint8_t *>(handle) + sizeof(h), &offset, sizeof(offset));
+    return MOE_OK;
+}
+
+int moe_ep_ipc_open(const void *handle, void **dev_ptr) {
+    if (!handle || !dev_ptr) return MOE_ERR_ARG;
+    cudaIpcMemHandle_t h;
+    uint64_t offset = 0;
+    std::memcpy(&h, handle, sizeof(h));
+    std::memcpy(&offset, static_cast<const uint8_t *>(handle) + sizeof(h), sizeof(offset));
+    void *base = nullptr;
+    if (cudaIpcOpenMemHandle(&base, h, cudaIpcMemLazyEnablePeerAccess) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    *dev_ptr = static_cast<uint8_t *>(base) + offset;
+    return MOE_OK;
+}
+
+int moe_ep_ipc_close(void *dev_ptr) {
+    if (!dev_ptr) return MOE_ERR_ARG;
+    auto range = moe::address_range_fn();
+    if (!range) return MOE_ERR_CUDA;
+    CUdeviceptr base = 0;
+    size_t size = 0;
+    if (range(&base, &size, reinterpret_cast<CUdeviceptr>(dev_ptr)) != CUDA_SUCCESS) return MOE_ERR_CUDA;
+    return cudaIpcCloseMemHandle(reinterpret_cast<void *>(base)) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 }  // extern "C"
