@@ -113,13 +113,19 @@ __device__ __forceinline__ TileCoord decode_tile(int t, int routed_tiles, const 
                                                  const int *s_tile_off) {
     TileCoord c;
     if (t < routed_tiles) {
-        const int mt = t / a.nb_r;
-        c.nb = t - mt * a.nb_r;
+        // Expert-major order: expert e owns tiles [tile_off[e] * nb_r, tile_off[e+1] * nb_r),
+        // n-block-major inside, so the m-tiles that read the same weight tile are
+        // neighbours in the round-robin and run at the same time (one HBM read,
+        // the others hit L2).
         int lo = 0, hi = a.E - 1;
         while (lo < hi) {
             const int mid = (lo + hi + 1) >> 1;
-            if (s_tile_off[mid] <= mt) lo = mid; else hi = mid - 1;
+            if (s_tile_off[mid] * a.nb_r <= t) lo = mid; else hi = mid - 1;
         }
+        const int mte = s_tile_off[lo + 1] - s_tile_off[lo];
+        const int local = t - s_tile_off[lo] * a.nb_r;
+        c.nb = local / mte;
+        const int mt = s_tile_off[lo] + (local - c.nb * mte);
         c.shared = false;
         c.e = lo;
         c.a_row = mt * GEMM_BM;
@@ -311,9 +317,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
                 const TileCoord c = decode_tile(t, routed_tiles, a, s_tile_off);
                 const CUtensorMap *mA = c.shared ? &mA_s : &mA_r;
-                // The n-blocks of one m-tile run on neighbouring CTAs and share the A
-                // tile; each starts at a different k-block so they do not all request
-                // the same lines at the same time.
+                // Tiles of one n-block (same weight tile) start at the same k-block and
+                // share each weight line as it arrives; the n-blocks of one m-tile
+                // (same token tile) start at different k-blocks, so they do not all
+                // request the same token lines at the same time.
                 const int rot = c.nb % c.kb;
                 for (int i = 0; i < c.kb; ++i, ++it) {
                     const int kb = i + rot < c.kb ? i + rot : i + rot - c.kb;
