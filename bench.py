@@ -300,11 +300,11 @@ def main():
     if cfg.N * cfg.k <= 2048:  # one fused dispatch kernel; its marks fill the first slot
         kernels = ["dispatch", "_", "_"] + kernels[3:]
 
-    def step(x):
-        moe.moe_router(x, inp.W_g, inp.b, cfg.n_group, cfg.topk_group, cfg.k, cfg.norm_topk_prob,
-                       cfg.alpha, idx, w, stream)
-        moe.moe_forward(x, inp.gate_up, inp.down, inp.sh_gate, inp.sh_up, inp.sh_down, idx, w, y,
-                        ws, stream)
+    def step(x, st=None):
+        # one library call: router, dispatch, experts, combine, shared expert
+        moe.moe_layer(x, inp.W_g, inp.b, inp.gate_up, inp.down, inp.sh_gate, inp.sh_up,
+                      inp.sh_down, cfg.n_group, cfg.topk_group, cfg.k, cfg.norm_topk_prob,
+                      cfg.alpha, ws, y, idx, w, stream if st is None else st)
 
     for _ in range(max(args.warmup, 3)):
         step(inp.x)
@@ -319,7 +319,9 @@ def main():
     reuse = float(loads.sum().item()) / max(hit, 1)
     routed_bytes_per_token = hit * 3.0 * cfg.D * cfg.d_moe * inp.gate_up.element_size() / cfg.N
 
-    # Per-step events: router start/end, then moe_forward's kernel boundaries.
+    # Per-step events at the layer call's kernel boundaries: start, after the router
+    # (which includes the dispatch and gather when they are fused into it), then
+    # after each later kernel.
     K = args.steps
     nk = len(kernels)
     # external=True: recorded as graph nodes when the steps are captured into a graph
@@ -333,13 +335,8 @@ def main():
     def timed_steps():
         st = torch.cuda.current_stream()  # the capture stream while a graph is captured
         for s_ in range(K):
-            row = evs[s_]
-            row[0].record(st)
-            moe.moe_router(inp.x, inp.W_g, inp.b, cfg.n_group, cfg.topk_group, cfg.k,
-                           cfg.norm_topk_prob, cfg.alpha, idx, w, st)
-            moe.moe_profile_set_events(row[1:])
-            moe.moe_forward(inp.x, inp.gate_up, inp.down, inp.sh_gate, inp.sh_up, inp.sh_down,
-                            idx, w, y, ws, st)
+            moe.moe_profile_set_events(evs[s_])
+            step(inp.x, st)
         moe.moe_profile_set_events([])
 
     # With --graph the K steps are captured once as a CUDA graph (kernel launches,

@@ -128,6 +128,24 @@ int moe_forward_clamped(const void *x, const void *gate_up, const void *down,
                         int d_moe, int d_sh, int k, int dtype, float gate_max, float up_max,
                         void *y, void *workspace, size_t ws_bytes, void *stream);
 
+/*
+ * moe_layer_forward — the whole layer in one call: moe_router then moe_forward
+ * ("GLM-4.5 Group Router" and "GLM-4.5 MoE Forward", How it works), with x's
+ * dtype `dtype` for the tokens and the experts and wg_dtype for W_g.  Writes
+ * topk_idx / topk_w (as moe_router) and y (as moe_forward); workspace as
+ * moe_forward (moe_forward_workspace bytes).  For a bf16 layer of at most 128
+ * tokens with at most 256 experts whose router runs on the tensor cores, the
+ * forward's dispatch and token gather run inside the router kernel (one cluster
+ * holds the whole routing), which saves two launches; the results are those of
+ * the two separate calls.  All arguments are checked before anything is
+ * launched; errors as moe_router and moe_forward.
+ */
+int moe_layer_forward(const void *x, const void *W_g, int wg_dtype, const float *b, int N, int D,
+                      int E, int n_group, int topk_group, int k, int norm_topk_prob, float alpha,
+                      const void *gate_up, const void *down, const void *sh_gate, const void *sh_up,
+                      const void *sh_down, int d_moe, int d_sh, int dtype, int32_t *topk_idx,
+                      float *topk_w, void *y, void *workspace, size_t ws_bytes, void *stream);
+
 /* Bytes of device scratch built into the library for moe_forward_noalloc. */
 #define MOE_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
 

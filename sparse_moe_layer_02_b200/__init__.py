@@ -41,7 +41,8 @@ MOE_EP_IPC_HANDLE_BYTES = 72
 EXPORTED_SYMBOLS = ("moe_router", "moe_forward_workspace", "moe_forward", "moe_device_status",
                     "moe_status_string", "moe_version", "moe_debug_set_wait_limit_ns",
                     "moe_debug_never_signal", "moe_profile_set_events", "moe_launch_count",
-                    "moe_forward_noalloc", "moe_forward_clamped", "moe_ep_symmetric_bytes",
+                    "moe_forward_noalloc", "moe_forward_clamped", "moe_layer_forward",
+                    "moe_ep_symmetric_bytes",
                     "moe_ep_workspace_bytes", "moe_ep_forward", "moe_ep_plan_host",
                     "moe_ep_ipc_export", "moe_ep_ipc_open", "moe_ep_ipc_close")
 
@@ -94,6 +95,9 @@ def load_library():
                                             P, ctypes.c_size_t, P]
         lib.moe_forward_clamped.restype = I
         S = ctypes.c_size_t
+        lib.moe_layer_forward.argtypes = [P, P, I, P, I, I, I, I, I, I, I, F, P, P, P, P, P, I, I, I,
+                                          P, P, P, P, S, P]
+        lib.moe_layer_forward.restype = I
         lib.moe_ep_symmetric_bytes.argtypes = [I, I, I, I, I]
         lib.moe_ep_symmetric_bytes.restype = S
         lib.moe_ep_workspace_bytes.argtypes = [I, I, I, I, I, I, I]
@@ -237,11 +241,35 @@ def moe_forward_noalloc(x, gate_up, down, sh_gate, sh_up, sh_down, topk_idx, top
 def moe_layer(x, W_g, b, gate_up, down, sh_gate, sh_up, sh_down, n_group, topk_group, k,
               norm_topk_prob, alpha, workspace=None, y=None, topk_idx=None, topk_w=None,
               stream=None):
-    """Whole layer: router then forward.  Returns (y, topk_idx, topk_w)."""
-    idx, w = moe_router(x, W_g, b, n_group, topk_group, k, norm_topk_prob, alpha, topk_idx,
-                        topk_w, stream)
-    y = moe_forward(x, gate_up, down, sh_gate, sh_up, sh_down, idx, w, y, workspace, stream)
-    return y, idx, w
+    """Whole layer in one library call (router then forward; small bf16 batches run the
+    dispatch inside the router kernel).  Returns (y, topk_idx, topk_w)."""
+    lib = load_library()
+    N, D = x.shape
+    E, two_d, D2 = gate_up.shape
+    d, d_sh = two_d // 2, sh_gate.shape[0]
+    if D2 != D or tuple(W_g.shape) != (E, D) or tuple(b.shape) != (E,) or b.dtype != torch.float32:
+        raise ValueError("inconsistent shapes")
+    dev = x.device
+    if topk_idx is None:
+        topk_idx = torch.empty((N, k), dtype=torch.int32, device=dev)
+    if topk_w is None:
+        topk_w = torch.empty((N, k), dtype=torch.float32, device=dev)
+    if y is None:
+        y = torch.empty((N, D), dtype=x.dtype, device=dev)
+    if workspace is None:
+        workspace = torch.empty(max(moe_forward_workspace(N, D, E, d, d_sh, k, x.dtype), 256),
+                                dtype=torch.uint8, device=dev)
+    if N == 0:
+        return y, topk_idx, topk_w
+    rc = lib.moe_layer_forward(_dev(x, "x"), _dev(W_g, "W_g"), _dt(W_g), _dev(b, "b"), N, D, E,
+                               n_group, topk_group, k, int(bool(norm_topk_prob)), float(alpha),
+                               _dev(gate_up, "gate_up"), _dev(down, "down"),
+                               _dev(sh_gate, "sh_gate"), _dev(sh_up, "sh_up"),
+                               _dev(sh_down, "sh_down"), d, d_sh, _dt(x), _dev(topk_idx, "topk_idx"),
+                               _dev(topk_w, "topk_w"), _dev(y, "y"), _dev(workspace, "workspace"),
+                               workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc, "moe_layer_forward")
+    return y, topk_idx, topk_w
 
 
 def moe_device_status(stream=None) -> int:

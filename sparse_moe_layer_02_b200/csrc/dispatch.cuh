@@ -160,21 +160,22 @@ __global__ void __launch_bounds__(DISPATCH_THREADS) dispatch_scatter_kernel(cons
 constexpr int DISPATCH_SMALL_IDS = 2048;
 constexpr int DISPATCH_SMALL_THREADS = 512;
 
-__global__ void __launch_bounds__(DISPATCH_SMALL_THREADS) dispatch_small_kernel(const DispatchParams p) {
-    constexpr int NW = DISPATCH_SMALL_THREADS / 32;
-    __shared__ int hist[DISPATCH_MAXE];
-    __shared__ int cursor[DISPATCH_MAXE];
-    __shared__ int wcnt[NW][DISPATCH_MAXE];
-    __shared__ int wsum[NW];
+// Body of the one-CTA dispatch for NT threads (NT >= E: thread e owns expert e in
+// the scan); shared arrays hist[DISPATCH_MAXE], cursor[DISPATCH_MAXE],
+// wcnt[NT/32][DISPATCH_MAXE], wsum[NT/32].
+template <int NT>
+__device__ __forceinline__ void dispatch_small_body(const DispatchParams &p, int *hist, int *cursor,
+                                                    int (*wcnt)[DISPATCH_MAXE], int *wsum) {
+    constexpr int NW = NT / 32;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int total = p.N * p.k;
-    for (int e = tid; e < p.E; e += DISPATCH_SMALL_THREADS) {
+    for (int e = tid; e < p.E; e += NT) {
         hist[e] = 0;
 #pragma unroll
         for (int w = 0; w < NW; ++w) wcnt[w][e] = 0;
     }
     __syncthreads();
-    for (int i = tid; i < total; i += DISPATCH_SMALL_THREADS) {
+    for (int i = tid; i < total; i += NT) {
         const int e = p.topk_idx[i];
         if (e >= 0 && e < p.E)
             atomicAdd(&hist[e], 1);
@@ -182,7 +183,7 @@ __global__ void __launch_bounds__(DISPATCH_SMALL_THREADS) dispatch_small_kernel(
             record_error(DEV_BAD_INDEX, 11);
     }
     __syncthreads();
-    // exclusive scan of tiles per expert (thread e owns expert e; E <= 512)
+    // exclusive scan of tiles per expert (thread e owns expert e; E <= NT)
     const int e = tid;
     const int cnt = e < p.E ? hist[e] : 0;
     const int tiles = (cnt + p.tile_rows - 1) / p.tile_rows;
@@ -218,9 +219,9 @@ __global__ void __launch_bounds__(DISPATCH_SMALL_THREADS) dispatch_small_kernel(
         p.meta[2] = incl;
     }
     __syncthreads();
-    // stable positions, DISPATCH_SMALL_THREADS ids per round
+    // stable positions, NT ids per round
     const uint32_t lt_mask = (1u << lane) - 1u;
-    for (int base = 0; base < total; base += DISPATCH_SMALL_THREADS) {
+    for (int base = 0; base < total; base += NT) {
         const int i = base + tid;
         const bool valid = i < total;
         int key = -1;
@@ -238,7 +239,7 @@ __global__ void __launch_bounds__(DISPATCH_SMALL_THREADS) dispatch_small_kernel(
             for (int w = 0; w < warp; ++w) pos += wcnt[w][key];
         }
         __syncthreads();
-        for (int ee = tid; ee < p.E; ee += DISPATCH_SMALL_THREADS) {
+        for (int ee = tid; ee < p.E; ee += NT) {
             int add = 0;
 #pragma unroll
             for (int w = 0; w < NW; ++w) {
@@ -258,6 +259,15 @@ __global__ void __launch_bounds__(DISPATCH_SMALL_THREADS) dispatch_small_kernel(
     }
 }
 
+__global__ void __launch_bounds__(DISPATCH_SMALL_THREADS) dispatch_small_kernel(const DispatchParams p) {
+    constexpr int NW = DISPATCH_SMALL_THREADS / 32;
+    __shared__ int hist[DISPATCH_MAXE];
+    __shared__ int cursor[DISPATCH_MAXE];
+    __shared__ int wcnt[NW][DISPATCH_MAXE];
+    __shared__ int wsum[NW];
+    dispatch_small_body<DISPATCH_SMALL_THREADS>(p, hist, cursor, wcnt, wsum);
+}
+
 // Copy each token's row of x to its k permuted rows (x_perm[pos_of[n, j]]).  A
 // warp takes one 2 KiB piece of one token's row: the piece is read once (x is
 // usually larger than L2, and the permuted order would otherwise re-read each row
@@ -265,38 +275,43 @@ __global__ void __launch_bounds__(DISPATCH_SMALL_THREADS) dispatch_small_kernel(
 // Padding rows stay unwritten: an MMA output row depends only on its own operand
 // row, and padding rows' outputs are never stored or read.  row_bytes is a
 // multiple of 16.
-__global__ void __launch_bounds__(256) dispatch_gather_kernel(const uint8_t *__restrict__ x,
-                                                              uint8_t *__restrict__ x_perm,
-                                                              const DispatchParams p,
-                                                              int row_bytes) {
+// One warp per item (token n, 2 KiB piece); items item0, item0 + step, ...
+__device__ __forceinline__ void gather_items(const uint8_t *__restrict__ x, uint8_t *__restrict__ x_perm,
+                                             const DispatchParams &p, int row_bytes, int item0,
+                                             int step) {
     const int lane = threadIdx.x & 31;
     const int nvec = row_bytes >> 4;
     const int pieces = (nvec + 127) / 128;
-    for (int item = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; item < p.N * pieces;
-         item += (gridDim.x * blockDim.x) >> 5) {
+    for (int item = item0; item < p.N * pieces; item += step) {
         const int n = item / pieces;
         const int v0 = (item - n * pieces) * 128;
         const int my_pos = lane < p.k ? p.pos_of[(size_t)n * p.k + lane] : -1;
         const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)n * row_bytes);
-        {
-            uint4 r[4];
+        uint4 r[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int v = v0 + lane + 32 * u;
+            if (v < nvec) r[u] = src[v];
+        }
+        for (int j = 0; j < p.k; ++j) {
+            const int pos = __shfl_sync(0xffffffffu, my_pos, j);
+            if (pos < 0) continue;
+            uint4 *dst = reinterpret_cast<uint4 *>(x_perm + (size_t)pos * row_bytes);
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 const int v = v0 + lane + 32 * u;
-                if (v < nvec) r[u] = src[v];
-            }
-            for (int j = 0; j < p.k; ++j) {
-                const int pos = __shfl_sync(0xffffffffu, my_pos, j);
-                if (pos < 0) continue;
-                uint4 *dst = reinterpret_cast<uint4 *>(x_perm + (size_t)pos * row_bytes);
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int v = v0 + lane + 32 * u;
-                    if (v < nvec) dst[v] = r[u];
-                }
+                if (v < nvec) dst[v] = r[u];
             }
         }
     }
+}
+
+__global__ void __launch_bounds__(256) dispatch_gather_kernel(const uint8_t *__restrict__ x,
+                                                              uint8_t *__restrict__ x_perm,
+                                                              const DispatchParams p,
+                                                              int row_bytes) {
+    gather_items(x, x_perm, p, row_bytes, (blockIdx.x * blockDim.x + threadIdx.x) >> 5,
+                 (gridDim.x * blockDim.x) >> 5);
 }
 
 }  // namespace moe

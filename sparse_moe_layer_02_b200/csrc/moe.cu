@@ -37,7 +37,8 @@ struct Profiler {
     cudaStream_t st;
     int next = 0;
     bool capturing = false;
-    explicit Profiler(cudaStream_t s) : st(s) {
+    explicit Profiler(cudaStream_t s, bool active = true) : st(s) {
+        if (!active) return;
         if (g_prof_n > 0) {
             cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
             capturing = cudaStreamIsCapturing(st, &cs) == cudaSuccess &&
@@ -232,7 +233,7 @@ int launch_router_x(const RouterParams &p, cudaStream_t st) {
 
 template <int EV, bool WF32>
 int launch_router_tc_t(const CUtensorMap &mX, const CUtensorMap &mW, const RouterParams &p, int clk,
-                       cudaStream_t st) {
+                       const RtcFuse &fz, cudaStream_t st) {
     constexpr int smem = RtcCfg<WF32>::SMEM;
     static int max_clk = 0; // largest cluster size this kernel can be launched with
     if (!max_clk) {
@@ -274,7 +275,7 @@ int launch_router_tc_t(const CUtensorMap &mX, const CUtensorMap &mW, const Route
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, router_tc_kernel<EV, WF32>, mX, mW, p, g_wait_limit_ns) !=
+    if (cudaLaunchKernelEx(&cfg, router_tc_kernel<EV, WF32>, mX, mW, p, g_wait_limit_ns, fz) !=
         cudaSuccess)
         return MOE_ERR_CUDA;
     return launch_status();
@@ -283,7 +284,7 @@ int launch_router_tc_t(const CUtensorMap &mX, const CUtensorMap &mW, const Route
 // Tensor-core router for bf16 x with a bf16 W_g (16 <= E <= 256) or an fp32 W_g
 // (16 <= E <= 192, three-way bf16 split); E % 16 == 0.
 template <bool WF32>
-int launch_router_tc(const RouterParams &p, int sms, cudaStream_t st) {
+int launch_router_tc(const RouterParams &p, int sms, const RtcFuse &fz, cudaStream_t st) {
     CUtensorMap mX, mW;
     if (!make_map(&mX, p.x, p.D, p.N, p.D, RTC_BM)) return MOE_ERR_CUDA;
     if (WF32) {
@@ -297,10 +298,10 @@ int launch_router_tc(const RouterParams &p, int sms, cudaStream_t st) {
     // device cannot co-schedule 16-CTA clusters of this kernel).
     int clk = 1;
     while (clk < RTC_MAX_CLK && 2 * clk * tblocks <= sms) clk *= 2;
-    if (p.E <= 32) return launch_router_tc_t<1, WF32>(mX, mW, p, clk, st);
-    if (p.E <= 64) return launch_router_tc_t<2, WF32>(mX, mW, p, clk, st);
-    if (p.E <= 128) return launch_router_tc_t<4, WF32>(mX, mW, p, clk, st);
-    return launch_router_tc_t<8, WF32>(mX, mW, p, clk, st);
+    if (p.E <= 32) return launch_router_tc_t<1, WF32>(mX, mW, p, clk, fz, st);
+    if (p.E <= 64) return launch_router_tc_t<2, WF32>(mX, mW, p, clk, fz, st);
+    if (p.E <= 128) return launch_router_tc_t<4, WF32>(mX, mW, p, clk, fz, st);
+    return launch_router_tc_t<8, WF32>(mX, mW, p, clk, fz, st);
 }
 
 template <int KIND>
@@ -371,6 +372,57 @@ int ensure_gemm_attrs(DeviceInfo *dev) {
     return MOE_OK;
 }
 
+// The router launch.  With fz (bf16 layers of at most 128 tokens whose logits run
+// on the tensor cores) the dispatch and gather of the forward run inside the
+// router kernel; *fused tells whether they did.
+int router_impl(const void *x, int x_dtype, const void *W_g, int wg_dtype, const float *b, int N,
+                int D, int E, int n_group, int topk_group, int k, int norm_topk_prob, float alpha,
+                int32_t *topk_idx, float *topk_w, void *stream, const RtcFuse *fz, bool *fused) {
+    if (fused) *fused = false;
+    int rc = check_router_shape(N, D, E, n_group, topk_group, k);
+    if (rc != MOE_OK) return rc;
+    if ((x_dtype != MOE_F32 && x_dtype != MOE_BF16) || (wg_dtype != MOE_F32 && wg_dtype != MOE_BF16))
+        return MOE_ERR_DTYPE;
+    if (N == 0) return MOE_OK;
+    if (!x || !W_g || !b || !topk_idx || !topk_w) return MOE_ERR_ARG;
+    if (!aligned16(x) || !aligned16(W_g) || !aligned16(b) || !aligned16(topk_idx) ||
+        !aligned16(topk_w))
+        return MOE_ERR_ARG;
+    DeviceInfo *dev = nullptr;
+    if ((rc = current_device_info(&dev)) != MOE_OK) return rc;
+    if (dev->major != 10) return MOE_ERR_NO_DEVICE;
+    RouterParams p;
+    p.x = x;
+    p.W_g = W_g;
+    p.b = b;
+    p.N = N;
+    p.D = D;
+    p.E = E;
+    p.G = n_group;
+    p.tg = topk_group;
+    p.k = k;
+    p.norm = norm_topk_prob ? 1 : 0;
+    p.alpha = alpha;
+    p.topk_idx = topk_idx;
+    p.topk_w = topk_w;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    RtcFuse off = {};
+    const bool tc = x_dtype == MOE_BF16 && E % 16 == 0 && E >= 16 && D % 8 == 0 &&
+                    ((wg_dtype == MOE_BF16 && E <= 256) || (wg_dtype == MOE_F32 && E <= RTC_MAXE_F32));
+    if (tc) {
+        const bool fuse = fz && fz->on && N <= RTC_BM && E <= RTC_THREADS;
+        if (fused) *fused = fuse;
+        const RtcFuse &f = fuse ? *fz : off;
+        return wg_dtype == MOE_BF16 ? launch_router_tc<false>(p, dev->sms, f, st)
+                                    : launch_router_tc<true>(p, dev->sms, f, st);
+    }
+    if (x_dtype == MOE_F32 && wg_dtype == MOE_F32) return launch_router_x<float, float>(p, st);
+    if (x_dtype == MOE_BF16 && wg_dtype == MOE_F32) return launch_router_x<__nv_bfloat16, float>(p, st);
+    if (x_dtype == MOE_BF16 && wg_dtype == MOE_BF16)
+        return launch_router_x<__nv_bfloat16, __nv_bfloat16>(p, st);
+    return launch_router_x<float, __nv_bfloat16>(p, st);
+}
+
 }  // namespace
 }  // namespace moe
 
@@ -417,42 +469,8 @@ unsigned long long moe_launch_count(void) { return g_launches.load(); }
 int moe_router(const void *x, int x_dtype, const void *W_g, int wg_dtype, const float *b, int N,
                int D, int E, int n_group, int topk_group, int k, int norm_topk_prob, float alpha,
                int32_t *topk_idx, float *topk_w, void *stream) {
-    int rc = check_router_shape(N, D, E, n_group, topk_group, k);
-    if (rc != MOE_OK) return rc;
-    if ((x_dtype != MOE_F32 && x_dtype != MOE_BF16) || (wg_dtype != MOE_F32 && wg_dtype != MOE_BF16))
-        return MOE_ERR_DTYPE;
-    if (N == 0) return MOE_OK;
-    if (!x || !W_g || !b || !topk_idx || !topk_w) return MOE_ERR_ARG;
-    if (!aligned16(x) || !aligned16(W_g) || !aligned16(b) || !aligned16(topk_idx) ||
-        !aligned16(topk_w))
-        return MOE_ERR_ARG;
-    DeviceInfo *dev = nullptr;
-    if ((rc = current_device_info(&dev)) != MOE_OK) return rc;
-    if (dev->major != 10) return MOE_ERR_NO_DEVICE;
-    RouterParams p;
-    p.x = x;
-    p.W_g = W_g;
-    p.b = b;
-    p.N = N;
-    p.D = D;
-    p.E = E;
-    p.G = n_group;
-    p.tg = topk_group;
-    p.k = k;
-    p.norm = norm_topk_prob ? 1 : 0;
-    p.alpha = alpha;
-    p.topk_idx = topk_idx;
-    p.topk_w = topk_w;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (x_dtype == MOE_BF16 && E % 16 == 0 && E >= 16 && D % 8 == 0) {
-        if (wg_dtype == MOE_BF16 && E <= 256) return launch_router_tc<false>(p, dev->sms, st);
-        if (wg_dtype == MOE_F32 && E <= RTC_MAXE_F32) return launch_router_tc<true>(p, dev->sms, st);
-    }
-    if (x_dtype == MOE_F32 && wg_dtype == MOE_F32) return launch_router_x<float, float>(p, st);
-    if (x_dtype == MOE_BF16 && wg_dtype == MOE_F32) return launch_router_x<__nv_bfloat16, float>(p, st);
-    if (x_dtype == MOE_BF16 && wg_dtype == MOE_BF16)
-        return launch_router_x<__nv_bfloat16, __nv_bfloat16>(p, st);
-    return launch_router_x<float, __nv_bfloat16>(p, st);
+    return moe::router_impl(x, x_dtype, W_g, wg_dtype, b, N, D, E, n_group, topk_group, k,
+                            norm_topk_prob, alpha, topk_idx, topk_w, stream, nullptr, nullptr);
 }
 
 size_t moe_forward_workspace(int N, int D, int E, int d_moe, int d_sh, int k, int dtype) {
@@ -466,18 +484,18 @@ size_t moe_forward_workspace(int N, int D, int E, int d_moe, int d_sh, int k, in
 namespace moe {
 namespace {
 
-int forward_impl(const void *x, const void *gate_up, const void *down, const void *sh_gate,
-                 const void *sh_up, const void *sh_down, const int32_t *topk_idx,
-                 const float *topk_w, int N, int D, int E, int d_moe, int d_sh, int k, int dtype,
-                 float gate_max, float up_max, void *y, void *workspace, size_t ws_bytes,
-                 void *stream) {
+// Validates the forward's arguments (nothing is launched on an error) and plans
+// its workspace.
+int check_forward(const void *x, const void *gate_up, const void *down, const void *sh_gate,
+                  const void *sh_up, const void *sh_down, const int32_t *topk_idx,
+                  const float *topk_w, int N, int D, int E, int d_moe, int d_sh, int k, int dtype,
+                  const void *y, const void *workspace, size_t ws_bytes, WsLayout &L) {
     if (dtype != MOE_F32 && dtype != MOE_BF16) return MOE_ERR_DTYPE;
     if (N < 0 || D <= 0 || E <= 0 || E > DISPATCH_MAXE || d_moe <= 0 || d_sh <= 0 || k <= 0 ||
         k > 32)
         return MOE_ERR_SHAPE;
     if (dtype == MOE_BF16 && (D % 8 || d_moe % 8 || d_sh % 8)) return MOE_ERR_SHAPE;
     if (dtype == MOE_F32 && (D % 4)) return MOE_ERR_SHAPE;
-    WsLayout L;
     if (!plan_workspace(N, D, E, d_moe, d_sh, k, dtype, L)) return MOE_ERR_SHAPE;
     if (N == 0) return MOE_OK;
     const void *ptrs[] = {x, gate_up, down, sh_gate, sh_up, sh_down, topk_idx, topk_w, y};
@@ -486,14 +504,12 @@ int forward_impl(const void *x, const void *gate_up, const void *down, const voi
     if (!workspace || !aligned16(workspace) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
         return MOE_ERR_WORKSPACE;
     if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
-    int rc;
-    DeviceInfo *dev = nullptr;
-    if ((rc = current_device_info(&dev)) != MOE_OK) return rc;
-    if (dev->major != 10) return MOE_ERR_NO_DEVICE;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    uint8_t *ws = static_cast<uint8_t *>(workspace);
-    Profiler prof(st);
+    return MOE_OK;
+}
 
+// Dispatch fields of the workspace (the same for the standalone and the fused dispatch).
+DispatchParams dispatch_params(const WsLayout &L, uint8_t *ws, const int32_t *topk_idx,
+                               const float *topk_w, int N, int k, int E) {
     DispatchParams dp;
     dp.topk_idx = topk_idx;
     dp.topk_w = topk_w;
@@ -509,8 +525,36 @@ int forward_impl(const void *x, const void *gate_up, const void *down, const voi
     dp.pos_of = reinterpret_cast<int32_t *>(ws + L.pos_of);
     dp.perm_tok = reinterpret_cast<int32_t *>(ws + L.perm_tok);
     dp.w_perm = reinterpret_cast<float *>(ws + L.w_perm);
+    return dp;
+}
 
-    if ((size_t)N * k <= DISPATCH_SMALL_IDS) {
+// The forward after routing.  prof_in: the caller's profiler (its marks continue);
+// dispatched: the router already ran the dispatch and gather (fused path).
+int forward_impl(const void *x, const void *gate_up, const void *down, const void *sh_gate,
+                 const void *sh_up, const void *sh_down, const int32_t *topk_idx,
+                 const float *topk_w, int N, int D, int E, int d_moe, int d_sh, int k, int dtype,
+                 float gate_max, float up_max, void *y, void *workspace, size_t ws_bytes,
+                 void *stream, Profiler *prof_in = nullptr, bool dispatched = false) {
+    WsLayout L;
+    int rc = check_forward(x, gate_up, down, sh_gate, sh_up, sh_down, topk_idx, topk_w, N, D, E,
+                           d_moe, d_sh, k, dtype, y, workspace, ws_bytes, L);
+    if (rc != MOE_OK || N == 0) return rc;
+    DeviceInfo *dev = nullptr;
+    if ((rc = current_device_info(&dev)) != MOE_OK) return rc;
+    if (dev->major != 10) return MOE_ERR_NO_DEVICE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    Profiler prof_own(st, prof_in == nullptr);
+    Profiler &prof = prof_in ? *prof_in : prof_own;
+
+    const DispatchParams dp = dispatch_params(L, ws, topk_idx, topk_w, N, k, E);
+
+    if (dispatched) {
+        // count, scan, scatter (and the gather below) ran inside the router kernel
+        prof.mark();
+        prof.mark();
+        prof.mark();
+    } else if ((size_t)N * k <= DISPATCH_SMALL_IDS) {
         // one CTA does count, scan and scatter (the three profiling marks coincide)
         dispatch_small_kernel<<<1, DISPATCH_SMALL_THREADS, 0, st>>>(dp);
         if ((rc = launched(prof)) != MOE_OK) return rc;
@@ -569,7 +613,9 @@ int forward_impl(const void *x, const void *gate_up, const void *down, const voi
 
     // ---- bf16 tensor-core path ----
     uint8_t *x_perm = ws + L.x_perm;
-    {
+    if (dispatched) {
+        prof.mark();
+    } else {
         const int items = N * ((D * 2 / 16 + 127) / 128); // 2 KiB pieces of token rows
         const int grid = std::min((items + 7) / 8, dev->sms * 16);
         dispatch_gather_kernel<<<grid, 256, 0, st>>>(static_cast<const uint8_t *>(x), x_perm, dp,
@@ -729,6 +775,43 @@ int moe_forward_clamped(const void *x, const void *gate_up, const void *down, co
     if (gate_max != gate_max || up_max != up_max || up_max < 0.f) return MOE_ERR_ARG;
     return forward_impl(x, gate_up, down, sh_gate, sh_up, sh_down, topk_idx, topk_w, N, D, E,
                         d_moe, d_sh, k, dtype, gate_max, up_max, y, workspace, ws_bytes, stream);
+}
+
+int moe_layer_forward(const void *x, const void *W_g, int wg_dtype, const float *b, int N, int D,
+                      int E, int n_group, int topk_group, int k, int norm_topk_prob, float alpha,
+                      const void *gate_up, const void *down, const void *sh_gate, const void *sh_up,
+                      const void *sh_down, int d_moe, int d_sh, int dtype, int32_t *topk_idx,
+                      float *topk_w, void *y, void *workspace, size_t ws_bytes, void *stream) {
+    using namespace moe;
+    int rc = check_router_shape(N, D, E, n_group, topk_group, k);
+    if (rc != MOE_OK) return rc;
+    if (wg_dtype != MOE_F32 && wg_dtype != MOE_BF16) return MOE_ERR_DTYPE;
+    WsLayout L;
+    if ((rc = check_forward(x, gate_up, down, sh_gate, sh_up, sh_down, topk_idx, topk_w, N, D, E,
+                            d_moe, d_sh, k, dtype, y, workspace, ws_bytes, L)) != MOE_OK)
+        return rc;
+    if (N == 0) return MOE_OK;
+    if (!W_g || !b || !aligned16(W_g) || !aligned16(b)) return MOE_ERR_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    Profiler prof(st);
+    // bf16 decode layers of one token block: dispatch and gather inside the router
+    RtcFuse fz = {};
+    if (dtype == MOE_BF16 && L.decode && (size_t)N * k <= DISPATCH_SMALL_IDS) {
+        fz.dp = dispatch_params(L, ws, topk_idx, topk_w, N, k, E);
+        fz.x = static_cast<const uint8_t *>(x);
+        fz.x_perm = ws + L.x_perm;
+        fz.row_bytes = D * 2;
+        fz.on = 1;
+    }
+    bool fused = false;
+    rc = router_impl(x, dtype, W_g, wg_dtype, b, N, D, E, n_group, topk_group, k, norm_topk_prob,
+                     alpha, topk_idx, topk_w, stream, &fz, &fused);
+    if (rc != MOE_OK) return rc;
+    prof.mark();
+    return forward_impl(x, gate_up, down, sh_gate, sh_up, sh_down, topk_idx, topk_w, N, D, E, d_moe,
+                        d_sh, k, dtype, INFINITY, INFINITY, y, workspace, ws_bytes, stream, &prof,
+                        fused);
 }
 
 int moe_device_status(void *stream) {

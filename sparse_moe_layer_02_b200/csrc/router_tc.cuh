@@ -22,6 +22,7 @@
 #include <cooperative_groups.h>
 
 #include "common.cuh"
+#include "dispatch.cuh"
 #include "router.cuh"
 
 namespace moe {
@@ -80,10 +81,23 @@ __device__ __forceinline__ void split_store(uint8_t *b0, int row, int chunk, con
     *reinterpret_cast<uint4 *>(b0 + 2 * part_bytes + off) = make_uint4(p3[0], p3[1], p3[2], p3[3]);
 }
 
+// Dispatch fused into the router for a batch of at most 128 tokens (one token
+// block, so one cluster holds the whole routing): after selection, CTA 0 of the
+// cluster runs the one-CTA dispatch on the routing just written, and then every
+// CTA of the cluster copies its share of the token rows into the expert-sorted
+// order.  on = 0: router only.
+struct RtcFuse {
+    DispatchParams dp;
+    const uint8_t *x;
+    uint8_t *x_perm;
+    int row_bytes;
+    int on;
+};
+
 template <int EV, bool WF32>
 __global__ void __launch_bounds__(RTC_THREADS, 1)
     router_tc_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mW,
-                     const RouterParams p, uint64_t limit) {
+                     const RouterParams p, uint64_t limit, const __grid_constant__ RtcFuse fz) {
     using C = RtcCfg<WF32>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -296,6 +310,23 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, tmem_cols);
+    }
+    if (fz.on) {
+        // The routing of all tokens is in global memory and visible to the whole
+        // cluster after the barrier above; the operand ring is free.
+        static_assert(RTC_THREADS / 32 * DISPATCH_MAXE * 4 + 3 * DISPATCH_MAXE * 4 <=
+                          RtcCfg<WF32>::STAGES * RtcCfg<WF32>::STAGE_BYTES,
+                      "dispatch arrays fit the ring");
+        if (rank == 0) {
+            int *hist = reinterpret_cast<int *>(ring);
+            int *cursor = hist + DISPATCH_MAXE;
+            int *wsum = cursor + DISPATCH_MAXE;
+            auto wcnt = reinterpret_cast<int(*)[DISPATCH_MAXE]>(wsum + DISPATCH_MAXE);
+            dispatch_small_body<RTC_THREADS>(fz.dp, hist, cursor, wcnt, wsum);
+        }
+        cluster.sync(); // positions visible to every CTA of the cluster
+        gather_items(fz.x, fz.x_perm, fz.dp, fz.row_bytes, rank * (RTC_THREADS / 32) + warp,
+                     CLK * (RTC_THREADS / 32));
     }
 }
 

@@ -90,3 +90,21 @@ def test_workspace_sizes():
     rows_max = (16384 * 8 + 127 * 256 + 127) // 128 * 128
     assert big > rows_max * 6144 * 2 * 2
     assert big < 6 * 2 ** 30
+
+
+def test_layer_call_rejects_bad_arguments_before_any_launch():
+    lib = moe.load_library()
+    call = lambda **kw: lib.moe_layer_forward(
+        16, kw.get("W_g", 16), kw.get("wdt", 1), 16, kw.get("N", 10), kw.get("D", 64),
+        kw.get("E", 16), kw.get("G", 1), kw.get("tg", 1), kw.get("k", 2), 1, 1.0, 16, 16, 16, 16,
+        16, kw.get("d", 32), 32, kw.get("dt", 1), 16, 16, 16, kw.get("ws", 256),
+        kw.get("wsb", 1 << 30), None)
+    assert call(G=3) == -2                 # router shape
+    assert call(k=40) == -2
+    assert call(wdt=7) == -3               # router dtype
+    assert call(dt=5) == -3                # forward dtype
+    assert call(d=20) == -2                # forward shape (bf16 rows of 16 bytes)
+    assert call(W_g=0) == -1               # null router matrix
+    assert call(ws=0) == -4
+    assert call(wsb=16) == -4
+    assert call(N=0) == 0                  # no-op

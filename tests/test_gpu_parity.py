@@ -286,3 +286,27 @@ def test_layer_parity_full_size_sampled(name):
     assert err["finite"] and err["max_rel"] <= Y_TOL[cfg.dtype]
     if cfg.skew:
         assert loads.max() / loads.mean() > 5.0
+
+
+# --------------------------------------------------------------- whole layer in one call
+@pytest.mark.parametrize("base,over", [
+    ("air_decode", {}),                      # fp32 W_g, 16-CTA router cluster, dispatch fused
+    ("glm5_decode", {}),                     # bf16 W_g, E = 256
+    ("air_decode", dict(N=1)),
+    ("air_decode", dict(N=128)),             # largest fused batch (one token block)
+    ("air_decode", dict(N=129)),             # two token blocks: separate dispatch kernels
+    ("skew_grouped", dict(N=64, D=512, E=64, n_group=8, topk_group=4, k=8, d_moe=256, d_sh=256,
+                          skew=False)),
+    ("glm5_prefill", dict(N=300, D=512, E=16, k=4, d_moe=256, d_sh=256)),
+])
+def test_layer_call_matches_router_then_forward(base, over):
+    cfg = CONFIGS[base].with_(**over) if over else CONFIGS[base]
+    inp = make_inputs(cfg, seed=2, device=DEV)
+    idx, w = moe.moe_router(inp.x, inp.W_g, inp.b, cfg.n_group, cfg.topk_group, cfg.k,
+                            cfg.norm_topk_prob, cfg.alpha)
+    y = moe.moe_forward(*_weights(inp), idx, w)
+    y2, idx2, w2 = moe.moe_layer(inp.x, inp.W_g, inp.b, *_weights(inp)[1:], cfg.n_group,
+                                 cfg.topk_group, cfg.k, cfg.norm_topk_prob, cfg.alpha)
+    assert moe.moe_device_status() == 0
+    assert torch.equal(idx, idx2) and torch.equal(w, w2)
+    assert torch.equal(y, y2)
