@@ -146,6 +146,22 @@ int moe_layer_forward(const void *x, const void *W_g, int wg_dtype, const float 
                       const void *sh_down, int d_moe, int d_sh, int dtype, int32_t *topk_idx,
                       float *topk_w, void *y, void *workspace, size_t ws_bytes, void *stream);
 
+/*
+ * moe_bias_update — one training step of the loss-free balancer on the router's
+ * correction bias ("GLM-4.5 Group Router", How it works: b is updated from expert
+ * load during training, at rate 0.001 for the first 15T tokens, then 0).  The page
+ * gives the rate, not the rule; this implements the plainest reading of the
+ * loss-free balancing it cites: with load_e the number of (token, slot) pairs of
+ * topk_idx [N, k] routed to expert e (the sentinel id E counts for nobody; other
+ * ids outside [0, E) are skipped and reported as MOE_ERR_BAD_INDEX by
+ * moe_device_status), every b_e (fp32, device, [E], updated in place) moves by
+ * `rate` towards the mean load: b_e += rate * sign(mean - load_e), decided exactly
+ * in integers.  loads_out (optional, [E] int32) receives the loads.  E <= 512.
+ * Errors: MOE_ERR_SHAPE, MOE_ERR_ARG (null b, NaN rate).
+ */
+int moe_bias_update(const int32_t *topk_idx, int N, int k, int E, float rate, float *b,
+                    int32_t *loads_out, void *stream);
+
 /* Bytes of device scratch built into the library for moe_forward_noalloc. */
 #define MOE_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
 

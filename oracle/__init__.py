@@ -16,6 +16,10 @@ G = 1 equals a full sort; brute-force enumeration on tiny group-routed inputs;
 sum(w) = alpha; w ratios equal s ratios (bias never in the weights);
 closed-form sigmoid and SwiGLU values; shared expert unscaled; sentinel skipped;
 the pages' parameter counts.
+
+``bias_update`` (the loss-free balancer's training step): parity unpinned.  The
+pages give its rate, not its rule; the function follows a stated reading, and
+its pins check that reading's properties, not values the pages print.
 """
 
 from __future__ import annotations
@@ -222,3 +226,26 @@ def param_counts(D: int, E: int, d: int, n_shared: int = 1, router_bias: bool = 
     router_p = E * D + (E if router_bias else 0)
     return {"expert": expert, "routed": E * expert, "shared": shared, "router": router_p,
             "block": E * expert + shared + router_p}
+
+
+def bias_update(idx, E: int, rate: float, b) -> tuple:
+    """One step of the loss-free balancer ("GLM-4.5 Group Router", How it works: the
+    bias b is updated from expert load during training, at rate 0.001 for the first
+    15T tokens, then 0).  The pages give the rate, not the rule; this follows the
+    plainest reading of the loss-free balancing they cite: every expert's bias moves
+    by `rate` towards the mean load, b_e += rate * sign(mean_load - load_e), with the
+    load counted over the routed (token, slot) pairs (the sentinel id E and any id
+    outside [0, E) count for nobody) and the comparison made exactly in integers
+    (sign(total - E * load_e)).  b is the fp32 buffer; the sum is taken in fp64 and
+    rounded once to fp32, as an fp32 add of rate would be.  Returns (b_new, loads).
+    parity unpinned: the rule is a reading, its pins check the reading's properties.
+    """
+    ids = np.asarray(idx).reshape(-1)
+    ids = ids[(ids >= 0) & (ids < E)]
+    loads = np.bincount(ids, minlength=E).astype(np.int64)
+    total = int(loads.sum())
+    sign = np.sign(total - E * loads).astype(np.float64)
+    b64 = np.asarray(torch.as_tensor(b).detach().cpu().float().numpy(), dtype=np.float64)
+    rate32 = float(np.float32(rate))
+    b_new = (b64 + rate32 * sign).astype(np.float32)
+    return b_new, loads

@@ -42,6 +42,7 @@ EXPORTED_SYMBOLS = ("moe_router", "moe_forward_workspace", "moe_forward", "moe_d
                     "moe_status_string", "moe_version", "moe_debug_set_wait_limit_ns",
                     "moe_debug_never_signal", "moe_profile_set_events", "moe_launch_count",
                     "moe_forward_noalloc", "moe_forward_clamped", "moe_layer_forward",
+                    "moe_bias_update",
                     "moe_ep_symmetric_bytes",
                     "moe_ep_workspace_bytes", "moe_ep_forward", "moe_ep_plan_host",
                     "moe_ep_ipc_export", "moe_ep_ipc_open", "moe_ep_ipc_close")
@@ -98,6 +99,8 @@ def load_library():
         lib.moe_layer_forward.argtypes = [P, P, I, P, I, I, I, I, I, I, I, F, P, P, P, P, P, I, I, I,
                                           P, P, P, P, S, P]
         lib.moe_layer_forward.restype = I
+        lib.moe_bias_update.argtypes = [P, I, I, I, F, P, P, P]
+        lib.moe_bias_update.restype = I
         lib.moe_ep_symmetric_bytes.argtypes = [I, I, I, I, I]
         lib.moe_ep_symmetric_bytes.restype = S
         lib.moe_ep_workspace_bytes.argtypes = [I, I, I, I, I, I, I]
@@ -270,6 +273,23 @@ def moe_layer(x, W_g, b, gate_up, down, sh_gate, sh_up, sh_down, n_group, topk_g
                                workspace.numel() * workspace.element_size(), _stream(stream))
     _check(rc, "moe_layer_forward")
     return y, topk_idx, topk_w
+
+
+def moe_bias_update(topk_idx, b, rate: float = 1e-3, loads=None, stream=None):
+    """One loss-free balancing step on the router bias b (fp32 [E], updated in place):
+    b_e += rate * sign(mean load - load_e) over the routing topk_idx [N, k].  Returns
+    (b, loads) with loads [E] int32 (allocated if not given)."""
+    if b.dtype != torch.float32 or b.dim() != 1:
+        raise ValueError("b must be a 1-D float32 tensor")
+    E = b.shape[0]
+    N, k = topk_idx.shape
+    if loads is None:
+        loads = torch.empty(E, dtype=torch.int32, device=b.device)
+    rc = load_library().moe_bias_update(_dev(topk_idx, "topk_idx") if N else 0, N, k, E,
+                                        float(rate), _dev(b, "b"), _dev(loads, "loads"),
+                                        _stream(stream))
+    _check(rc, "moe_bias_update")
+    return b, loads
 
 
 def moe_device_status(stream=None) -> int:

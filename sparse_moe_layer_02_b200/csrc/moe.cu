@@ -473,6 +473,21 @@ int moe_router(const void *x, int x_dtype, const void *W_g, int wg_dtype, const 
                             norm_topk_prob, alpha, topk_idx, topk_w, stream, nullptr, nullptr);
 }
 
+int moe_bias_update(const int32_t *topk_idx, int N, int k, int E, float rate, float *b,
+                    int32_t *loads_out, void *stream) {
+    if (N < 0 || k <= 0 || k > 32 || E <= 0 || E > 512) return MOE_ERR_SHAPE;
+    if ((size_t)N * k > (size_t)INT32_MAX) return MOE_ERR_SHAPE;
+    if (rate != rate) return MOE_ERR_ARG;
+    if (!b || (N > 0 && !topk_idx)) return MOE_ERR_ARG;
+    int rc;
+    moe::DeviceInfo *dev = nullptr;
+    if ((rc = moe::current_device_info(&dev)) != MOE_OK) return rc;
+    if (dev->major != 10) return MOE_ERR_NO_DEVICE;
+    moe::bias_update_kernel<<<1, moe::BIAS_THREADS, 0, static_cast<cudaStream_t>(stream)>>>(
+        topk_idx, N * k, E, rate, b, loads_out);
+    return moe::launch_status();
+}
+
 size_t moe_forward_workspace(int N, int D, int E, int d_moe, int d_sh, int k, int dtype) {
     WsLayout L;
     if (!plan_workspace(N, D, E, d_moe, d_sh, k, dtype, L)) return 0;

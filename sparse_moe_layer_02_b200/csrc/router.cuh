@@ -175,6 +175,43 @@ __device__ __forceinline__ void router_select(const RouterParams &p, int t, cons
     }
 }
 
+// One step of the loss-free balancer ("GLM-4.5 Group Router", How it works: the
+// bias is updated from expert load during training, at rate 0.001, then 0).  The
+// rule is the plainest reading of the loss-free balancing the page cites: every
+// expert's bias moves by `rate` towards the mean load, b_e += rate * sign(mean -
+// load_e), the comparison made exactly in integers (total - E * load_e).  Loads
+// count the routed (token, slot) pairs; the sentinel E counts for nobody, other
+// out-of-range ids are reported.  One CTA of BIAS_THREADS threads, E <= 512.
+constexpr int BIAS_THREADS = 512;
+
+__global__ void __launch_bounds__(BIAS_THREADS)
+    bias_update_kernel(const int32_t *topk_idx, int n_ids, int E, float rate, float *b,
+                       int32_t *loads_out) {
+    __shared__ int hist[512];
+    __shared__ long long total;
+    for (int e = threadIdx.x; e < E; e += BIAS_THREADS) hist[e] = 0;
+    if (threadIdx.x == 0) total = 0;
+    __syncthreads();
+    int mine = 0;
+    for (int i = threadIdx.x; i < n_ids; i += BIAS_THREADS) {
+        const int e = topk_idx[i];
+        if (e >= 0 && e < E) {
+            atomicAdd(&hist[e], 1);
+            ++mine;
+        } else if (e != E) {
+            record_error(DEV_BAD_INDEX, 12);
+        }
+    }
+    atomicAdd(reinterpret_cast<unsigned long long *>(&total), (unsigned long long)mine);
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += BIAS_THREADS) {
+        const long long diff = total - (long long)E * hist[e];
+        const float step = diff > 0 ? rate : (diff < 0 ? -rate : 0.f);
+        b[e] = b[e] + step;
+        if (loads_out) loads_out[e] = hist[e];
+    }
+}
+
 // EV = experts per lane (E <= 32 * EV); each thread accumulates 4 tokens x EV experts.
 template <typename XT, typename WT, int EV>
 __global__ void __launch_bounds__(ROUTER_THREADS)

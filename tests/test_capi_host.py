@@ -108,3 +108,12 @@ def test_layer_call_rejects_bad_arguments_before_any_launch():
     assert call(ws=0) == -4
     assert call(wsb=16) == -4
     assert call(N=0) == 0                  # no-op
+
+
+def test_bias_update_rejects_bad_arguments():
+    lib = moe.load_library()
+    assert lib.moe_bias_update(None, 4, 2, 600, 1e-3, 16, None, None) == -2      # E > 512
+    assert lib.moe_bias_update(None, 4, 0, 16, 1e-3, 16, None, None) == -2       # k
+    assert lib.moe_bias_update(None, 4, 2, 16, float("nan"), 16, None, None) == -1
+    assert lib.moe_bias_update(None, 4, 2, 16, 1e-3, None, None, None) == -1     # null b
+    assert lib.moe_bias_update(None, 4, 2, 16, 1e-3, 16, None, None) == -1       # null ids

@@ -310,3 +310,20 @@ def test_layer_call_matches_router_then_forward(base, over):
     assert moe.moe_device_status() == 0
     assert torch.equal(idx, idx2) and torch.equal(w, w2)
     assert torch.equal(y, y2)
+
+
+# --------------------------------------------------------------- loss-free bias update
+@pytest.mark.parametrize("N,k,E,rate", [(64, 4, 16, 1e-3), (4096, 8, 256, 1e-3), (1, 8, 128, 0.5),
+                                        (16384, 8, 160, 1e-3), (0, 8, 64, 1e-3)])
+def test_bias_update_matches_oracle(N, k, E, rate):
+    g = torch.Generator().manual_seed(N + E)
+    idx = torch.randint(0, E, (N, k), generator=g, dtype=torch.int32)
+    if N:
+        idx[0, 0] = E                                  # a sentinel counts for nobody
+    b = (torch.rand(E, generator=g) - 0.5) * 0.1
+    b_ref, loads_ref = oracle.bias_update(idx.numpy(), E, rate, b)
+    b_d = b.to(DEV)
+    _, loads = moe.moe_bias_update(idx.to(DEV), b_d, rate)
+    assert moe.moe_device_status() == 0
+    np.testing.assert_array_equal(loads.cpu().numpy(), loads_ref)
+    np.testing.assert_array_equal(b_d.cpu().numpy(), b_ref)          # bit-exact
