@@ -37,7 +37,7 @@ UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 BF16_KERNELS = ["dispatch_count", "dispatch_scan", "dispatch_scatter", "dispatch_gather",
-                "gate_up_swiglu", "down_combine_shared"]
+                "gate_up_swiglu", "down_combine_shared", "combine"]
 F32_KERNELS = ["dispatch_count", "dispatch_scan", "dispatch_scatter", "gate_up_routed",
                "gate_up_shared", "down_routed", "down_shared", "combine"]
 
@@ -191,6 +191,9 @@ def kernel_work(cfg, name: str, hit: int):
     elif name == "down_combine_shared":
         flops = 2.0 * (N * k * d + N * dsh) * D
         byts = (hit * d + dsh) * D * es + N * D * es
+    elif name == "combine":  # prefill: k slot rows and the fp32 shared row in, y out
+        flops = 0.0
+        byts = N * k * D * es + N * D * 4 + N * D * es
     elif name == "router":
         flops = 2.0 * N * D * E
         byts = E * D * ws + N * D * es

@@ -210,10 +210,10 @@ int moe_version(void);
  * Test hooks for the bounded device-side waits (no GPU fault is involved).
  *   moe_debug_set_wait_limit_ns: limit for every spin-wait in the kernels
  *     (default 2e9 ns); ns = 0 restores the default.
- *   moe_debug_never_signal: when on, the shared-expert combine of the next
- *     moe_forward calls waits for one more routed tile than exists, so the wait
- *     runs out, the status word reports MOE_ERR_DEVICE_TIMEOUT and the kernel
- *     returns normally.
+ *   moe_debug_never_signal: when on, the combine of the next moe_forward calls
+ *     (the decode down kernel's shared tiles, or the prefill combine kernel)
+ *     waits for one more expert tile than exists, so the wait runs out, the
+ *     status word reports MOE_ERR_DEVICE_TIMEOUT and the kernel returns normally.
  */
 int moe_debug_set_wait_limit_ns(uint64_t ns);
 int moe_debug_never_signal(int on);

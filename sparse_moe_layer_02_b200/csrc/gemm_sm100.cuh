@@ -91,6 +91,7 @@ struct GemmArgs {
     uint64_t wait_limit_ns;
     int never_signal;
     float gate_max, up_max; // gate_up: SwiGLU limits (+infinity = plain SwiGLU)
+    int no_combine;         // down: leave the combine to combine_kernel (launched next)
     // Expert parallelism (all null / 0 for a single-device layer).  The routed
     // rows are other ranks' tokens received into this rank's buffer.
     const uint32_t *ep_wait_ctr;    // gate_up: rows arrived (this epoch) ...
@@ -231,6 +232,35 @@ __device__ __forceinline__ void combine_rows(const GemmArgs &a, int gwarp, int n
             }
         }
     }
+}
+
+// The combine as its own launch after the down kernel (which then skips its final
+// phase): many more warps per SM than the persistent GEMM's six keep many more
+// slot loads in flight.  Same rows, same order of adds as the in-kernel phase.
+constexpr int COMBINE_THREADS = 256;
+
+__global__ void __launch_bounds__(COMBINE_THREADS) combine_kernel(const GemmArgs g) {
+    constexpr int W = COMBINE_THREADS / 32;
+    // Every down tile has been counted (the launch follows the down kernel on the
+    // stream, so this holds at once; the bounded check reports a tile that never
+    // completed instead of combining stale slots).
+    __shared__ int failed;
+    if (threadIdx.x == 0) {
+        failed = 0;
+        const int target = g.meta[2] * g.nb_r + g.mt_s * g.nb_s + (g.never_signal ? 1 : 0);
+        const uint64_t t0 = globaltimer_ns();
+        while (ld_acquire_gpu(&g.meta[0]) < target) {
+            if (globaltimer_ns() - t0 > g.wait_limit_ns) {
+                record_error(DEV_TIMEOUT, 122);
+                failed = 1;
+                break;
+            }
+            __nanosleep(256);
+        }
+    }
+    __syncthreads();
+    if (failed) return;
+    combine_rows(g, blockIdx.x * W + (threadIdx.x >> 5), gridDim.x * W, threadIdx.x & 31);
 }
 
 template <int KIND>
@@ -507,7 +537,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         tmem_dealloc(tmem_base, GEMM_TMEM_COLS);
     }
 
-    if (KIND == GEMM_DOWN && a.ep_P == 0) {
+    if (KIND == GEMM_DOWN && a.ep_P == 0 && !a.no_combine) {
         // ---- combine phase: every tile of the launch must be stored first ----------
         if (threadIdx.x == 0 && !*abort_flag) {
             const int target = total_tiles + (a.never_signal ? 1 : 0);

@@ -699,6 +699,7 @@ int forward_impl(const void *x, const void *gate_up, const void *down, const voi
         rc = launch_decode<GEMM_DOWN>(mdn, mh_perm, msd, msd, mh_sh, g,
                                       std::min(dev->sms, max_tiles), true, st);
         prof.mark();
+        prof.mark(); // the combine ran inside the down kernel
         return rc;
     }
 
@@ -762,11 +763,15 @@ int forward_impl(const void *x, const void *gate_up, const void *down, const voi
     g.pos_of = dp.pos_of;
     g.slot = slot;
     g.osh = reinterpret_cast<float *>(ws + L.osh);
+    g.no_combine = 1;
     max_tiles = mt_r_max * g.nb_r + mt_s * g.nb_s;
     rc = launch_gemm<GEMM_DOWN>(mh_perm, mdn, mh_sh, msd, msd, g, std::min(dev->sms, max_tiles),
-                                true, st);
+                                false, st);
     prof.mark();
-    return rc;
+    if (rc != MOE_OK) return rc;
+    // y = slots in slot order + shared output, at many warps per SM
+    combine_kernel<<<std::min((N + 7) / 8, dev->sms * 8), COMBINE_THREADS, 0, st>>>(g);
+    return launched(prof);
 }
 
 }  // namespace
