@@ -43,9 +43,15 @@ constexpr int GEMM_B_BYTES = GEMM_BN * GEMM_BK * 2;  // 32 KiB
 constexpr int GEMM_STAGE_BYTES = GEMM_A_BYTES + GEMM_B_BYTES;
 constexpr int GEMM_TMEM_COLS = 512;
 constexpr int GEMM_MAXE = 512;
-// Shared memory: 1024 alignment slack + ring + barriers/flags + tile table.
-constexpr int GEMM_SMEM_BYTES =
-    1024 + GEMM_STAGES * GEMM_STAGE_BYTES + 256 + (GEMM_MAXE + 1) * 4 + 64;
+// Shared memory: 1024 alignment slack + ring + barriers/flags + tile table, then
+// (1024-aligned) the down epilogue's store staging: per epilogue warp two buffers
+// of 32 rows x 32 bf16 columns.
+constexpr int GEMM_OUT_BOX = 32;                                   // rows and columns of a store box
+constexpr int GEMM_OUT_BUF = GEMM_OUT_BOX * GEMM_OUT_BOX * 2;     // 2 KiB
+constexpr int GEMM_STG_OFF =
+    (GEMM_STAGES * GEMM_STAGE_BYTES + 256 + (GEMM_MAXE + 1) * 4 + 1023) / 1024 * 1024;
+constexpr int GEMM_SMEM_BYTES = 1024 + GEMM_STG_OFF + 4 * 2 * GEMM_OUT_BUF;
+static_assert(GEMM_SMEM_BYTES <= 232448, "shared memory");
 
 enum GemmKind { GEMM_GATE_UP = 0, GEMM_DOWN = 1 };
 
@@ -92,6 +98,7 @@ struct GemmArgs {
     int never_signal;
     float gate_max, up_max; // gate_up: SwiGLU limits (+infinity = plain SwiGLU)
     int no_combine;         // down: leave the combine to combine_kernel (launched next)
+    int tma_out;            // down: routed rows stored by TMA through the mOut map
     // Expert parallelism (all null / 0 for a single-device layer).  The routed
     // rows are other ranks' tokens received into this rank's buffer.
     const uint32_t *ep_wait_ctr;    // gate_up: rows arrived (this epoch) ...
@@ -263,13 +270,15 @@ __global__ void __launch_bounds__(COMBINE_THREADS) combine_kernel(const GemmArgs
     combine_rows(g, blockIdx.x * W + (threadIdx.x >> 5), gridDim.x * W, threadIdx.x & 31);
 }
 
+// mOut (down with tma_out): the slot rows [rows, D] bf16, box 32 x 32, no swizzle.
 template <int KIND>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap mA_r,
                         const __grid_constant__ CUtensorMap mB_r,
                         const __grid_constant__ CUtensorMap mA_s,
                         const __grid_constant__ CUtensorMap mB_s0,
-                        const __grid_constant__ CUtensorMap mB_s1, const GemmArgs a) {
+                        const __grid_constant__ CUtensorMap mB_s1,
+                        const __grid_constant__ CUtensorMap mOut, const GemmArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -427,6 +436,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         const int q = warp & 3;          // TMEM lane quadrant of this warp
         const int row = q * 32 + lane;   // row of the tile owned by this thread
         const int ep_tid = threadIdx.x - 64;
+        uint8_t *stg = smem + GEMM_STG_OFF + q * 2 * GEMM_OUT_BUF; // this warp's two store buffers
+        uint32_t nstore = 0;             // store boxes this warp has staged
         uint32_t tc = 0;
         for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++tc) {
             const TileCoord c = decode_tile(t, routed_tiles, a, s_tile_off);
@@ -464,6 +475,48 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                             h[i] = swiglu_f(__uint_as_float(g[i]), __uint_as_float(u[i]),
                                             a.gate_max, a.up_max);
                         store_row_chunk_bf16(row_ptr, col, ncols, h);
+                    }
+                }
+            } else if (!c.shared && a.tma_out) {
+                // Routed rows are contiguous in the slot buffer: each 32-column chunk
+                // of this warp's 32 rows is staged in shared memory and written by
+                // one TMA store (full lines, off the epilogue threads' critical path).
+                const float wr = a.w_perm[c.a_row + row];
+#pragma unroll 1
+                for (int ch = 0; ch < 8; ++ch) {
+                    uint32_t v[32];
+                    tmem_ld_32x32b_x32(tbase + ch * 32, v);
+                    tmem_ld_wait();
+                    const int col = c.nb * GEMM_BN + ch * 32;
+                    if (col < a.ncols_r) {
+                        uint8_t *buf = stg + (nstore & 1) * GEMM_OUT_BUF;
+                        if (lane == 0) bulk_wait_group_read<1>(); // the box staged 2 ago left buf
+                        __syncwarp();
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            pk[i] = pack_bf16x2(wr * __uint_as_float(v[2 * i]),
+                                                wr * __uint_as_float(v[2 * i + 1]));
+                        const uint4 u[4] = {make_uint4(pk[0], pk[1], pk[2], pk[3]),
+                                            make_uint4(pk[4], pk[5], pk[6], pk[7]),
+                                            make_uint4(pk[8], pk[9], pk[10], pk[11]),
+                                            make_uint4(pk[12], pk[13], pk[14], pk[15])};
+                        uint4 *dst = reinterpret_cast<uint4 *>(buf + lane * (GEMM_OUT_BOX * 2));
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            // rotate the pieces across lanes (fewer bank conflicts); the
+                            // selects keep the data in registers
+                            const int p = (j + lane) & 3;
+                            const uint4 val = p == 0 ? u[0] : p == 1 ? u[1] : p == 2 ? u[2] : u[3];
+                            dst[p] = val;
+                        }
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_2d(&mOut, buf, col, c.a_row + q * 32);
+                            bulk_commit_group();
+                        }
+                        ++nstore;
                     }
                 }
             } else if (!c.shared) {
@@ -530,6 +583,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         }
     }
 
+    if (KIND == GEMM_DOWN && warp >= 2 && lane == 0) bulk_wait_group<0>(); // stores done
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {

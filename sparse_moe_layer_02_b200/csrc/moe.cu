@@ -184,6 +184,21 @@ bool make_map(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows, ui
     return r == CUDA_SUCCESS;
 }
 
+// 2-D bf16 map for TMA stores of the down epilogue: box 32 columns x 32 rows,
+// no swizzle (the staging buffer holds the box row-major).
+bool make_map_out(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows, uint64_t ld) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {ld * 2};
+    cuuint32_t box[2] = {GEMM_OUT_BOX, GEMM_OUT_BOX};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 int launch_status() {
     g_launches.fetch_add(1, std::memory_order_relaxed);
     const cudaError_t e = cudaGetLastError();
@@ -306,8 +321,8 @@ int launch_router_tc(const RouterParams &p, int sms, const RtcFuse &fz, cudaStre
 
 template <int KIND>
 int launch_gemm(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &a2,
-                const CUtensorMap &a3, const CUtensorMap &a4, const GemmArgs &args, int grid,
-                bool cooperative, cudaStream_t st) {
+                const CUtensorMap &a3, const CUtensorMap &a4, const CUtensorMap &a5,
+                const GemmArgs &args, int grid, bool cooperative, cudaStream_t st) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid, 1, 1);
     cfg.blockDim = dim3(GEMM_THREADS, 1, 1);
@@ -318,7 +333,7 @@ int launch_gemm(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap 
     attr[0].val.cooperative = cooperative ? 1 : 0;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<KIND>, a0, a1, a2, a3, a4, args) !=
+    if (cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<KIND>, a0, a1, a2, a3, a4, a5, args) !=
         cudaSuccess)
         return MOE_ERR_CUDA;
     return launch_status();
@@ -742,8 +757,8 @@ int forward_impl(const void *x, const void *gate_up, const void *down, const voi
     g.ld_s = d_sh;
     g.ncols_s = d_sh;
     int max_tiles = mt_r_max * g.nb_r + mt_s * g.nb_s;
-    rc = launch_gemm<GEMM_GATE_UP>(mx_perm, mgu, mx, msg, msu, g, std::min(dev->sms, max_tiles),
-                                   false, st);
+    rc = launch_gemm<GEMM_GATE_UP>(mx_perm, mgu, mx, msg, msu, mx, g,
+                                   std::min(dev->sms, max_tiles), false, st);
     prof.mark();
     if (rc != MOE_OK) return rc;
 
@@ -764,9 +779,12 @@ int forward_impl(const void *x, const void *gate_up, const void *down, const voi
     g.slot = slot;
     g.osh = reinterpret_cast<float *>(ws + L.osh);
     g.no_combine = 1;
+    g.tma_out = 1;
+    CUtensorMap mslot;
+    if (!make_map_out(&mslot, slot, D, L.rows_max, D)) return MOE_ERR_CUDA;
     max_tiles = mt_r_max * g.nb_r + mt_s * g.nb_s;
-    rc = launch_gemm<GEMM_DOWN>(mh_perm, mdn, mh_sh, msd, msd, g, std::min(dev->sms, max_tiles),
-                                false, st);
+    rc = launch_gemm<GEMM_DOWN>(mh_perm, mdn, mh_sh, msd, msd, mslot, g,
+                                std::min(dev->sms, max_tiles), false, st);
     prof.mark();
     if (rc != MOE_OK) return rc;
     // y = slots in slot order + shared output, at many warps per SM
@@ -1038,8 +1056,8 @@ int ep_forward_impl(int phases, int P, int rank, uint32_t epoch, void *const *pe
         g.ep_wait_ctr = reinterpret_cast<const uint32_t *>(own + S.ctr) + par;
         g.ep_wait_target = ep.rmeta + 3;
         int max_tiles = mt_r_max * g.nb_r + mt_s * g.nb_s;
-        rc = launch_gemm<GEMM_GATE_UP>(mx_perm, mgu, mx, msg, msu, g, std::min(dev->sms, max_tiles),
-                                       false, st);
+        rc = launch_gemm<GEMM_GATE_UP>(mx_perm, mgu, mx, msg, msu, mx, g,
+                                       std::min(dev->sms, max_tiles), false, st);
         prof.mark();
         if (rc != MOE_OK) return rc;
         g.ep_wait_ctr = nullptr;
@@ -1061,8 +1079,8 @@ int ep_forward_impl(int phases, int P, int rank, uint32_t epoch, void *const *pe
             g.ep_ret[q] = reinterpret_cast<uint32_t *>(ep.sym[q] + S.ctr) + 2 + par;
         }
         max_tiles = mt_r_max * g.nb_r + mt_s * g.nb_s;
-        rc = launch_gemm<GEMM_DOWN>(mh_perm, mdn, mh_sh, msd, msd, g, std::min(dev->sms, max_tiles),
-                                    true, st);
+        rc = launch_gemm<GEMM_DOWN>(mh_perm, mdn, mh_sh, msd, msd, msd, g,
+                                    std::min(dev->sms, max_tiles), true, st);
         prof.mark();
         if (rc != MOE_OK) return rc;
     }

@@ -47,9 +47,6 @@ template <bool WF32> struct RtcCfg {
                   "partial logits reuse the operand ring");
 };
 
-__device__ __forceinline__ void fence_proxy_async_smem() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
 
 // Split 8 fp32 router weights into three bf16 parts, written as one 16-byte chunk
 // of each part's K-major tile with the 128-byte swizzle the MMA descriptor uses.
