@@ -97,7 +97,6 @@ struct GemmArgs {
     uint64_t wait_limit_ns;
     int never_signal;
     float gate_max, up_max; // gate_up: SwiGLU limits (+infinity = plain SwiGLU)
-    int no_combine;         // down: leave the combine to combine_kernel (launched next)
     int tma_out;            // down: routed rows stored by TMA through the mOut map
     // Expert parallelism (all null / 0 for a single-device layer).  The routed
     // rows are other ranks' tokens received into this rank's buffer.
@@ -181,8 +180,8 @@ __device__ __forceinline__ void acc_bf16x8(float (&acc)[8], const uint4 &w) {
 // y[n] = sum_{j<k} slot[pos(n, j)] (slot order) + osh[n], one warp per row, each
 // lane four 8-column pieces at a time.  The slot rows are fetched eight slots at
 // a time before any of them is added, so 32 slot loads and the shared row are in
-// flight per lane (the phase is bound by load latency at one CTA of six warps per
-// SM); the adds then run in slot order (a missing slot adds +0).
+// flight per lane (the loop is bound by load latency); the adds then run in slot
+// order (a missing slot adds +0).
 __device__ __forceinline__ void combine_rows(const GemmArgs &a, int gwarp, int nwarps, int lane) {
     constexpr int U = 4;
     const int pieces = a.ncols_s / 8;
@@ -290,7 +289,6 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     uint64_t *drain = tempty + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    volatile int *combine_failed = abort_flag + 1;
     int *s_tile_off = reinterpret_cast<int *>(smem + GEMM_STAGES * GEMM_STAGE_BYTES + 256);
 
     const int warp = warp_id(), lane = lane_id();
@@ -306,7 +304,6 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
-        *combine_failed = 0;
         fence_mbar_init();
     }
     if (warp == 0 && lane == 0) {
@@ -575,7 +572,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             if (lane == 0) mbar_arrive(&tempty[acc]);
             }  // have
             if (KIND == GEMM_DOWN) {
-                // Publish this tile's stores to the combine phase.
+                // Count the finished tile (combine_kernel checks the count).
                 __threadfence();
                 named_bar_sync(1, 128);
                 if (ep_tid == 0 && have) atomicAdd(&a.meta[0], 1);
@@ -589,25 +586,6 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, GEMM_TMEM_COLS);
-    }
-
-    if (KIND == GEMM_DOWN && a.ep_P == 0 && !a.no_combine) {
-        // ---- combine phase: every tile of the launch must be stored first ----------
-        if (threadIdx.x == 0 && !*abort_flag) {
-            const int target = total_tiles + (a.never_signal ? 1 : 0);
-            const uint64_t t0 = globaltimer_ns();
-            while (ld_acquire_gpu(&a.meta[0]) < target) {
-                if (globaltimer_ns() - t0 > limit) {
-                    record_error(DEV_TIMEOUT, 120);
-                    *combine_failed = 1;
-                    break;
-                }
-                __nanosleep(256);
-            }
-        }
-        __syncthreads();
-        if (!*combine_failed && !*abort_flag) combine_rows(a, blockIdx.x * (GEMM_THREADS / 32) + warp,
-                                                           gridDim.x * (GEMM_THREADS / 32), lane);
     }
 }
 

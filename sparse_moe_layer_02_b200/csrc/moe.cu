@@ -778,7 +778,6 @@ int forward_impl(const void *x, const void *gate_up, const void *down, const voi
     g.pos_of = dp.pos_of;
     g.slot = slot;
     g.osh = reinterpret_cast<float *>(ws + L.osh);
-    g.no_combine = 1;
     g.tma_out = 1;
     CUtensorMap mslot;
     if (!make_map_out(&mslot, slot, D, L.rows_max, D)) return MOE_ERR_CUDA;
