@@ -107,7 +107,7 @@ int check_router_shape(int N, int D, int E, int G, int tg, int k) {
 // ---------------------------------------------------------------------------
 struct WsLayout {
     size_t chunk_hist, counts, tile_off, meta, pos_of, perm_tok, w_perm;
-    size_t x_perm, h_perm, h_sh, slot, osh, total;
+    size_t x_perm, h_perm, h_sh, slot, osh, wg_parts, total;
     int nchunks;
     size_t rows_max;
     bool decode;
@@ -146,6 +146,8 @@ bool plan_workspace(int N, int D, int E, int d, int d_sh, int k, int dtype, WsLa
     L.slot = take(L.rows_max * D * es);
     // fp32 output of the shared expert, combined with the slots (prefill kernels)
     L.osh = take(dtype == MOE_BF16 && !L.decode ? (size_t)N * D * 4 : 0);
+    // the router matrix split into three bf16 parts (moe_layer_forward, fp32 W_g)
+    L.wg_parts = take((size_t)3 * E * D * 2);
     L.total = off;
     return true;
 }
@@ -302,7 +304,10 @@ template <bool WF32>
 int launch_router_tc(const RouterParams &p, int sms, const RtcFuse &fz, cudaStream_t st) {
     CUtensorMap mX, mW;
     if (!make_map(&mX, p.x, p.D, p.N, p.D, RTC_BM)) return MOE_ERR_CUDA;
-    if (WF32) {
+    if (WF32 && p.wg_parts) {
+        // the three bf16 parts [3E, D]; a box is one part's E rows
+        if (!make_map(&mW, p.wg_parts, p.D, 3 * (uint64_t)p.E, p.D, p.E)) return MOE_ERR_CUDA;
+    } else if (WF32) {
         mW = mX; // unused: the fp32 matrix is read and split by the kernel's own warps
     } else if (!make_map(&mW, p.W_g, p.D, p.E, p.D, p.E)) {
         return MOE_ERR_CUDA;
@@ -390,9 +395,12 @@ int ensure_gemm_attrs(DeviceInfo *dev) {
 // The router launch.  With fz (bf16 layers of at most 128 tokens whose logits run
 // on the tensor cores) the dispatch and gather of the forward run inside the
 // router kernel; *fused tells whether they did.
+// wg_parts_ws: optional scratch of 3 * E * D bf16 for splitting an fp32 W_g once per
+// call (used when the batch has several token blocks).
 int router_impl(const void *x, int x_dtype, const void *W_g, int wg_dtype, const float *b, int N,
                 int D, int E, int n_group, int topk_group, int k, int norm_topk_prob, float alpha,
-                int32_t *topk_idx, float *topk_w, void *stream, const RtcFuse *fz, bool *fused) {
+                int32_t *topk_idx, float *topk_w, void *stream, const RtcFuse *fz, bool *fused,
+                void *wg_parts_ws = nullptr) {
     if (fused) *fused = false;
     int rc = check_router_shape(N, D, E, n_group, topk_group, k);
     if (rc != MOE_OK) return rc;
@@ -420,6 +428,7 @@ int router_impl(const void *x, int x_dtype, const void *W_g, int wg_dtype, const
     p.alpha = alpha;
     p.topk_idx = topk_idx;
     p.topk_w = topk_w;
+    p.wg_parts = nullptr;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     RtcFuse off = {};
     const bool tc = x_dtype == MOE_BF16 && E % 16 == 0 && E >= 16 && D % 8 == 0 &&
@@ -427,6 +436,15 @@ int router_impl(const void *x, int x_dtype, const void *W_g, int wg_dtype, const
     if (tc) {
         const bool fuse = fz && fz->on && N <= RTC_BM && E <= RTC_THREADS;
         if (fused) *fused = fuse;
+        if (wg_dtype == MOE_F32 && wg_parts_ws && N > RTC_BM) {
+            // split W_g once instead of in every token block
+            const size_t n8 = (size_t)E * D / 8;
+            const int grid = (int)std::min<size_t>((n8 + 255) / 256, (size_t)dev->sms * 8);
+            wg_split_kernel<<<grid, 256, 0, st>>>(static_cast<const float *>(W_g), E, D,
+                                                  static_cast<__nv_bfloat16 *>(wg_parts_ws));
+            if ((rc = launch_status()) != MOE_OK) return rc;
+            p.wg_parts = wg_parts_ws;
+        }
         const RtcFuse &f = fuse ? *fz : off;
         return wg_dtype == MOE_BF16 ? launch_router_tc<false>(p, dev->sms, f, st)
                                     : launch_router_tc<true>(p, dev->sms, f, st);
@@ -843,7 +861,7 @@ int moe_layer_forward(const void *x, const void *W_g, int wg_dtype, const float 
     }
     bool fused = false;
     rc = router_impl(x, dtype, W_g, wg_dtype, b, N, D, E, n_group, topk_group, k, norm_topk_prob,
-                     alpha, topk_idx, topk_w, stream, &fz, &fused);
+                     alpha, topk_idx, topk_w, stream, &fz, &fused, ws + L.wg_parts);
     if (rc != MOE_OK) return rc;
     prof.mark();
     return forward_impl(x, gate_up, down, sh_gate, sh_up, sh_down, topk_idx, topk_w, N, D, E, d_moe,

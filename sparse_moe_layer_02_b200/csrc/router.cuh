@@ -35,6 +35,9 @@ struct RouterParams {
     float alpha;
     int32_t *topk_idx;
     float *topk_w;
+    // fp32 W_g already split into three bf16 parts [3][E][D] (null: the tensor-core
+    // router splits it itself, per token block)
+    const void *wg_parts;
 };
 
 // Dynamic shared memory of router_kernel<EV>: x chunk, W chunk, partial logits,

@@ -48,10 +48,10 @@ template <bool WF32> struct RtcCfg {
 };
 
 
-// Split 8 fp32 router weights into three bf16 parts, written as one 16-byte chunk
-// of each part's K-major tile with the 128-byte swizzle the MMA descriptor uses.
-__device__ __forceinline__ void split_store(uint8_t *b0, int row, int chunk, const float4 &u,
-                                            const float4 &v, int part_bytes) {
+// Split 8 fp32 router weights into three bf16 parts w = w1 + w2 + w3 (each part
+// packed as 8 bf16 in a uint4).
+__device__ __forceinline__ void split8(const float4 &u, const float4 &v, uint4 &q1, uint4 &q2,
+                                       uint4 &q3) {
     const float w[8] = {u.x, u.y, u.z, u.w, v.x, v.y, v.z, v.w};
     uint32_t p1[4], p2[4], p3[4];
 #pragma unroll
@@ -72,10 +72,41 @@ __device__ __forceinline__ void split_store(uint8_t *b0, int row, int chunk, con
         p2[h] = pack_bf16x2(a2[0], a2[1]);
         p3[h] = pack_bf16x2(a3[0], a3[1]);
     }
+    q1 = make_uint4(p1[0], p1[1], p1[2], p1[3]);
+    q2 = make_uint4(p2[0], p2[1], p2[2], p2[3]);
+    q3 = make_uint4(p3[0], p3[1], p3[2], p3[3]);
+}
+
+// The three parts of 8 weights written as one 16-byte chunk of each part's K-major
+// tile with the 128-byte swizzle the MMA descriptor uses.
+__device__ __forceinline__ void split_store(uint8_t *b0, int row, int chunk, const float4 &u,
+                                            const float4 &v, int part_bytes) {
+    uint4 q1, q2, q3;
+    split8(u, v, q1, q2, q3);
     const int off = row * 128 + ((chunk ^ (row & 7)) << 4);
-    *reinterpret_cast<uint4 *>(b0 + off) = make_uint4(p1[0], p1[1], p1[2], p1[3]);
-    *reinterpret_cast<uint4 *>(b0 + part_bytes + off) = make_uint4(p2[0], p2[1], p2[2], p2[3]);
-    *reinterpret_cast<uint4 *>(b0 + 2 * part_bytes + off) = make_uint4(p3[0], p3[1], p3[2], p3[3]);
+    *reinterpret_cast<uint4 *>(b0 + off) = q1;
+    *reinterpret_cast<uint4 *>(b0 + part_bytes + off) = q2;
+    *reinterpret_cast<uint4 *>(b0 + 2 * part_bytes + off) = q3;
+}
+
+// The same split of the whole fp32 W_g [E][D] into parts [3][E][D] in global memory,
+// once per call, for batches of several token blocks: the router then loads the
+// three parts by TMA instead of splitting them again in every token block.
+// D % 8 == 0; one thread per 8 weights.
+__global__ void __launch_bounds__(256) wg_split_kernel(const float *__restrict__ W, int E, int D,
+                                                       __nv_bfloat16 *__restrict__ parts) {
+    const size_t n8 = (size_t)E * D / 8;
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n8;
+         i += (size_t)gridDim.x * blockDim.x) {
+        const float4 u = __ldg(reinterpret_cast<const float4 *>(W) + 2 * i);
+        const float4 v = __ldg(reinterpret_cast<const float4 *>(W) + 2 * i + 1);
+        uint4 q1, q2, q3;
+        split8(u, v, q1, q2, q3);
+        uint4 *out = reinterpret_cast<uint4 *>(parts);
+        out[i] = q1;
+        out[n8 + i] = q2;
+        out[2 * n8 + i] = q3;
+    }
 }
 
 // Dispatch fused into the router for a batch of at most 128 tokens (one token
@@ -125,9 +156,10 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
     auto kb_of = [&](int i) { return kb0 + (i + rot < nkb ? i + rot : i + rot - nkb); };
     constexpr int NCONV = 6; // warps 2-7 split fp32 W_g
 
+    const bool presplit = WF32 && p.wg_parts != nullptr; // the three parts come by TMA (mW)
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
-            mbar_init(&full[s], WF32 ? 1 + NCONV : 1);
+            mbar_init(&full[s], WF32 && !presplit ? 1 + NCONV : 1);
             mbar_init(&empty[s], 1);
         }
         mbar_init(tfull, 1);
@@ -136,7 +168,7 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
     }
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&mX);
-        if (!WF32) tma_prefetch_desc(&mW);
+        if (!WF32 || presplit) tma_prefetch_desc(&mW);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, tmem_cols);
@@ -156,9 +188,14 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
                 const uint32_t s = it % C::STAGES, ph = (it / C::STAGES) & 1;
                 if (!mbar_wait(&empty[s], ph ^ 1, limit, abort_flag, 300)) { ok = false; break; }
                 uint8_t *sa = ring + s * C::STAGE_BYTES;
-                mbar_arrive_expect_tx(&full[s], RTC_A_BYTES + (WF32 ? 0u : (uint32_t)E * RTC_BK * 2));
+                const uint32_t wbytes = (uint32_t)E * RTC_BK * 2;
+                mbar_arrive_expect_tx(&full[s], RTC_A_BYTES + (!WF32 ? wbytes : presplit ? 3 * wbytes : 0u));
                 tma_load_2d(&mX, &full[s], sa, kb * RTC_BK, t0);
                 if (!WF32) tma_load_2d(&mW, &full[s], sa + RTC_A_BYTES, kb * RTC_BK, 0);
+                if (presplit)
+                    for (int part_i = 0; part_i < 3; ++part_i)
+                        tma_load_2d(&mW, &full[s], sa + RTC_A_BYTES + part_i * C::B_PART, kb * RTC_BK,
+                                    part_i * E);
             }
             if (!ok) {
                 const uint32_t first = it > (uint32_t)C::STAGES ? it - C::STAGES : 0;
@@ -192,7 +229,7 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
             umma_commit(tfull); // arrives once every MMA issued above has completed
         }
         __syncwarp();
-    } else if (WF32) {
+    } else if (WF32 && !presplit) {
         // Split fp32 W_g into three bf16 tiles per stage (warps 2-7).  A thread owns
         // up to SPLIT_IT 8-float pieces of a k-block.  The next k-block's pieces are
         // loaded into registers while the current ones are split and stored, so the

@@ -298,6 +298,8 @@ def test_layer_parity_full_size_sampled(name):
     ("skew_grouped", dict(N=64, D=512, E=64, n_group=8, topk_group=4, k=8, d_moe=256, d_sh=256,
                           skew=False)),
     ("glm5_prefill", dict(N=300, D=512, E=16, k=4, d_moe=256, d_sh=256)),
+    # fp32 W_g over several token blocks: W_g is split once, not in every block
+    ("glm45_prefill", dict(N=300, D=520, E=48, k=4, d_moe=256, d_sh=256)),
 ])
 def test_layer_call_matches_router_then_forward(base, over):
     cfg = CONFIGS[base].with_(**over) if over else CONFIGS[base]
