@@ -20,13 +20,13 @@
 // the routed tiles in the same launch.
 //
 // down: one tile = 128 rows x 256 output columns of W_down (D x d_moe).  Routed
-// tiles scale each row by its routing weight and store a bf16 per-slot partial;
-// the shared expert's tiles store their fp32 output.  Every tile then bumps a
-// done counter.  When a CTA has no tiles left it waits (bounded) for the counter
-// to cover every tile of the launch, and then all CTAs of the same persistent
-// launch combine: row n of y = the k slot partials summed in slot order plus the
-// shared expert's output at scale 1, written once in bf16 (deterministic: no
-// atomics on the output), one warp per row with 16-byte loads.
+// tiles scale each row by its routing weight; each epilogue warp stages 32 rows x
+// 32 columns of bf16 per-slot partials in shared memory and writes them with one
+// TMA store (the permuted rows of a tile are contiguous in the slot buffer).  The
+// shared expert's tiles store their fp32 output.  Every tile bumps a done counter.
+// The combine is the next launch (combine_kernel): row n of y = the k slot
+// partials summed in slot order plus the shared expert's output at scale 1,
+// written once in bf16 (deterministic: no atomics on the output).
 #pragma once
 
 #include "common.cuh"
@@ -240,9 +240,9 @@ __device__ __forceinline__ void combine_rows(const GemmArgs &a, int gwarp, int n
     }
 }
 
-// The combine as its own launch after the down kernel (which then skips its final
-// phase): many more warps per SM than the persistent GEMM's six keep many more
-// slot loads in flight.  Same rows, same order of adds as the in-kernel phase.
+// The combine, launched after the down kernel: one warp per row of y (see
+// combine_rows).  As the down kernel's own final phase (six warps per SM) it ran
+// 0.26-0.64 ms slower on the prefill workloads.
 constexpr int COMBINE_THREADS = 256;
 
 __global__ void __launch_bounds__(COMBINE_THREADS) combine_kernel(const GemmArgs g) {
@@ -547,7 +547,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 }
                 if (a.ep_P > 0) warp_count_rows(a.ep_ret, src, a.ep_P);
             } else {
-                // shared expert: fp32 output rows, combined after every tile is done
+                // shared expert: fp32 output rows, added last by combine_kernel
                 const int n = c.a_row + row;
                 float *row_ptr = a.osh + (size_t)n * a.ld_s;
 #pragma unroll 1
