@@ -24,7 +24,7 @@ __all__ = ["MoEError", "moe_router", "moe_forward", "moe_forward_workspace", "mo
            "EXPORTED_SYMBOLS", "moe_ep_symmetric_bytes", "moe_ep_workspace_bytes",
            "moe_ep_forward", "moe_ep_plan_host", "moe_ep_ipc_export", "moe_ep_ipc_open",
            "moe_ep_ipc_close", "ExpertParallelGroup", "MOE_EP_COUNT", "MOE_EP_SEND",
-           "MOE_EP_EXPERTS", "MOE_EP_COMBINE", "MOE_EP_ALL"]
+           "MOE_EP_EXPERTS", "MOE_EP_COMBINE", "MOE_EP_ALL", "moe_bias_update"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libmoe.so")
