@@ -306,9 +306,10 @@ def moe_debug_never_signal(on: bool):
 
 
 def moe_profile_set_events(events) -> None:
-    """Record the given torch.cuda.Event objects at moe_forward's kernel boundaries
-    (events[0] before the first kernel, events[i] after the i-th); [] turns it off."""
-    handles = [int(e.cuda_event) for e in events]
+    """Record the given torch.cuda.Event objects at the next calls' kernel boundaries
+    (events[0] before the first kernel, events[i] after the i-th; None skips a
+    boundary); [] turns it off."""
+    handles = [int(e.cuda_event) if e is not None else 0 for e in events]
     arr = (ctypes.c_void_p * max(len(handles), 1))(*handles)
     _check(load_library().moe_profile_set_events(arr, len(handles)), "moe_profile_set_events")
 
