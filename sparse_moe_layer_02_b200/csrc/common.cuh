@@ -102,7 +102,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64
 // ---------------------------------------------------------------------------
 // TMA: 2-D tiled bulk tensor load global -> shared, completion on an mbarrier.
 // c0 is the innermost (contiguous) coordinate in elements, c1 the row.
-// No multicast form is used anywhere in this library.
+// Every TMA load in this library fills only the issuing CTA's own shared memory.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void tma_load_2d(const CUtensorMap *map, uint64_t *bar, void *dst,
                                             int c0, int c1) {
