@@ -129,6 +129,9 @@ SMALL = {
     "bf16_decode_multitile": ("glm5_decode", dict(N=250, D=256, E=4, k=2, d_moe=128, d_sh=64)),
     "bf16_decode_group": ("skew_grouped", dict(N=64, D=384, E=64, n_group=8, topk_group=4, k=8,
                                                d_moe=192, d_sh=320, skew=False)),
+    # the limits: E = 512 experts (CUDA-core router), k = 32 experts per token
+    "bf16_max_experts": ("glm5_prefill", dict(N=300, D=256, E=512, k=32, d_moe=64, d_sh=64)),
+    "bf16_decode_max_experts": ("glm5_decode", dict(N=64, D=256, E=512, k=32, d_moe=64, d_sh=64)),
     # n_shared_experts = 3: one shared MLP of width 3 d_moe
     "bf16_n_shared3": ("glm5_prefill", dict(N=300, D=256, E=8, k=4, d_moe=128, d_sh=384)),
     "bf16_decode_n_shared3": ("glm5_decode", dict(N=48, D=256, E=8, k=4, d_moe=128, d_sh=384)),
