@@ -213,15 +213,23 @@ int launched(Profiler &prof) {
     return rc;
 }
 
+int current_device_index() {
+    int dev = 0;
+    return cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < kMaxDevices ? dev : -1;
+}
+
 template <typename XT, typename WT, int EV>
 int launch_router_t(const RouterParams &p, cudaStream_t st) {
     constexpr int smem = router_smem_bytes(EV);
-    static bool attr_set = false; // per process; the attribute is per function
-    if (!attr_set) {
+    static bool attr_set[kMaxDevices] = {}; // function attributes are set per device
+    const int dev = current_device_index();
+    if (dev < 0) return MOE_ERR_CUDA;
+    if (!attr_set[dev]) {
+        std::lock_guard<std::mutex> lk(g_mu);
         if (cudaFuncSetAttribute(router_kernel<XT, WT, EV>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
             return MOE_ERR_CUDA;
-        attr_set = true;
+        attr_set[dev] = true;
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(ROUTER_CL, (p.N + ROUTER_TM - 1) / ROUTER_TM, 1);
@@ -252,8 +260,14 @@ template <int EV, bool WF32>
 int launch_router_tc_t(const CUtensorMap &mX, const CUtensorMap &mW, const RouterParams &p, int clk,
                        const RtcFuse &fz, cudaStream_t st) {
     constexpr int smem = RtcCfg<WF32>::SMEM;
-    static int max_clk = 0; // largest cluster size this kernel can be launched with
+    // largest cluster size this kernel can be launched with, per device (the
+    // attributes are set per device)
+    static int max_clk_of[kMaxDevices] = {};
+    const int dev = current_device_index();
+    if (dev < 0) return MOE_ERR_CUDA;
+    int &max_clk = max_clk_of[dev];
     if (!max_clk) {
+        std::lock_guard<std::mutex> lk(g_mu);
         if (cudaFuncSetAttribute(router_tc_kernel<EV, WF32>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
             return MOE_ERR_CUDA;
