@@ -280,7 +280,7 @@ __global__ void __launch_bounds__(256) ep_send_kernel(const EpParams p) {
 
 // combine phase: wait (bounded) until every row this rank's pairs get back has
 // been stored, then y = sum of the k slots in slot order + shared output.
-__global__ void __launch_bounds__(256) ep_combine_kernel(const EpParams p, const GemmArgs g) {
+__global__ void __launch_bounds__(256, 2) ep_combine_kernel(const EpParams p, const GemmArgs g) {
     __shared__ int fail;
     if (threadIdx.x == 0) {
         fail = 0;

@@ -178,12 +178,14 @@ __device__ __forceinline__ void acc_bf16x8(float (&acc)[8], const uint4 &w) {
 }
 
 // y[n] = sum_{j<k} slot[pos(n, j)] (slot order) + osh[n], one warp per row, each
-// lane four 8-column pieces at a time.  The slot rows are fetched eight slots at
-// a time before any of them is added, so 32 slot loads and the shared row are in
+// lane U 8-column pieces at a time.  The slot rows are fetched eight slots at a
+// time before any of them is added, so 8 U slot loads and the shared row are in
 // flight per lane (the loop is bound by load latency); the adds then run in slot
-// order (a missing slot adds +0).
+// order (a missing slot adds +0).  U = 2 keeps a thread at 128 registers, so two
+// 256-thread CTAs fit on an SM; with U = 4 (228 registers, one CTA per SM) the
+// combine ran 20-26 % slower.
+template <int U = 2>
 __device__ __forceinline__ void combine_rows(const GemmArgs &a, int gwarp, int nwarps, int lane) {
-    constexpr int U = 4;
     const int pieces = a.ncols_s / 8;
     for (int n = gwarp; n < a.N; n += nwarps) {
         const int my_pos = lane < a.k ? a.pos_of[(size_t)n * a.k + lane] : -1;
@@ -245,7 +247,7 @@ __device__ __forceinline__ void combine_rows(const GemmArgs &a, int gwarp, int n
 // 0.26-0.64 ms slower on the prefill workloads.
 constexpr int COMBINE_THREADS = 256;
 
-__global__ void __launch_bounds__(COMBINE_THREADS) combine_kernel(const GemmArgs g) {
+__global__ void __launch_bounds__(COMBINE_THREADS, 2) combine_kernel(const GemmArgs g) {
     constexpr int W = COMBINE_THREADS / 32;
     // Every down tile has been counted (the launch follows the down kernel on the
     // stream, so this holds at once; the bounded check reports a tile that never

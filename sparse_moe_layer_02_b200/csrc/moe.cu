@@ -819,7 +819,7 @@ int forward_impl(const void *x, const void *gate_up, const void *down, const voi
     prof.mark();
     if (rc != MOE_OK) return rc;
     // y = slots in slot order + shared output, at many warps per SM
-    combine_kernel<<<std::min((N + 7) / 8, dev->sms * 8), COMBINE_THREADS, 0, st>>>(g);
+    combine_kernel<<<std::min((N + 7) / 8, dev->sms * 16), COMBINE_THREADS, 0, st>>>(g);
     return launched(prof);
 }
 
