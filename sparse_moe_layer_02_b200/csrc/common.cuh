@@ -253,11 +253,6 @@ template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16
     return __bfloat162float(v);
 }
 
-template <typename T> __device__ __forceinline__ T from_f32(float v);
-template <> __device__ __forceinline__ float from_f32<float>(float v) { return v; }
-template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) {
-    return __float2bfloat16_rn(v);
-}
 
 // SiLU(a) = a * sigmoid(a), with the fast exponential.
 __device__ __forceinline__ float silu_f(float a) { return a / (1.0f + __expf(-a)); }
