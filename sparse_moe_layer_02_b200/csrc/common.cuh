@@ -148,6 +148,17 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
+// Programmatic dependent launch.  A grid launched with programmatic stream
+// serialization may start before the previous kernel in its stream has finished;
+// grid_dep_wait() returns once that kernel has completed and its memory writes are
+// visible (at once for a grid launched without the attribute).
+// grid_dep_launch_dependents() lets the next such grid in the stream start
+// launching its CTAs (which then wait in their own grid_dep_wait()).
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------------------
 // tcgen05: shared-memory matrix descriptor for a K-major operand tile written
 // by TMA with 128-byte swizzle: rows of 128 bytes (64 bf16), 8-row core groups

@@ -154,6 +154,10 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
         if (KIND == GEMM_GATE_UP) tma_prefetch_desc(&mA_s1);
         tma_prefetch_desc(&mB_s);
     }
+    // Nothing above reads or writes global memory or TMEM, so it may overlap the
+    // previous kernel of the stream (programmatic launch); everything below follows it.
+    grid_dep_wait();
+    grid_dep_launch_dependents();
     if (warp == 1) {
         tmem_alloc(tmem_slot, DEC_TMEM_COLS);
         tmem_relinquish();

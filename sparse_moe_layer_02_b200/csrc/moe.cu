@@ -218,6 +218,20 @@ int current_device_index() {
     return cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < kMaxDevices ? dev : -1;
 }
 
+// cudaLaunchKernelEx; a launch refused with the programmatic-serialization attribute
+// (always the last one) is repeated without it.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_ex(cudaLaunchConfig_t cfg, void (*kernel)(KArgs...), Args &&...args) {
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
+    if (e != cudaSuccess && cfg.numAttrs > 0 &&
+        cfg.attrs[cfg.numAttrs - 1].id == cudaLaunchAttributeProgrammaticStreamSerialization) {
+        cudaGetLastError();
+        --cfg.numAttrs;
+        e = cudaLaunchKernelEx(&cfg, kernel, args...);
+    }
+    return e;
+}
+
 template <typename XT, typename WT, int EV>
 int launch_router_t(const RouterParams &p, cudaStream_t st) {
     constexpr int smem = router_smem_bytes(EV);
@@ -258,7 +272,7 @@ int launch_router_x(const RouterParams &p, cudaStream_t st) {
 
 template <int EV, bool WF32>
 int launch_router_tc_t(const CUtensorMap &mX, const CUtensorMap &mW, const RouterParams &p, int clk,
-                       const RtcFuse &fz, cudaStream_t st) {
+                       const RtcFuse &fz, bool pdl, cudaStream_t st) {
     constexpr int smem = RtcCfg<WF32>::SMEM;
     // largest cluster size this kernel can be launched with, per device (the
     // attributes are set per device)
@@ -299,23 +313,25 @@ int launch_router_tc_t(const CUtensorMap &mX, const CUtensorMap &mW, const Route
     cfg.blockDim = dim3(RTC_THREADS, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = clk;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, router_tc_kernel<EV, WF32>, mX, mW, p, g_wait_limit_ns, fz) !=
-        cudaSuccess)
+    cfg.numAttrs = pdl ? 2 : 1;
+    if (launch_ex(cfg, router_tc_kernel<EV, WF32>, mX, mW, p, g_wait_limit_ns, fz) != cudaSuccess)
         return MOE_ERR_CUDA;
     return launch_status();
 }
 
 // Tensor-core router for bf16 x with a bf16 W_g (16 <= E <= 256) or an fp32 W_g
 // (16 <= E <= 192, three-way bf16 split); E % 16 == 0.
+// pdl: launch with programmatic stream serialization (the fused decode path).
 template <bool WF32>
-int launch_router_tc(const RouterParams &p, int sms, const RtcFuse &fz, cudaStream_t st) {
+int launch_router_tc(const RouterParams &p, int sms, const RtcFuse &fz, bool pdl, cudaStream_t st) {
     CUtensorMap mX, mW;
     if (!make_map(&mX, p.x, p.D, p.N, p.D, RTC_BM)) return MOE_ERR_CUDA;
     if (WF32 && p.wg_parts) {
@@ -332,10 +348,10 @@ int launch_router_tc(const RouterParams &p, int sms, const RtcFuse &fz, cudaStre
     // device cannot co-schedule 16-CTA clusters of this kernel).
     int clk = 1;
     while (clk < RTC_MAX_CLK && 2 * clk * tblocks <= sms) clk *= 2;
-    if (p.E <= 32) return launch_router_tc_t<1, WF32>(mX, mW, p, clk, fz, st);
-    if (p.E <= 64) return launch_router_tc_t<2, WF32>(mX, mW, p, clk, fz, st);
-    if (p.E <= 128) return launch_router_tc_t<4, WF32>(mX, mW, p, clk, fz, st);
-    return launch_router_tc_t<8, WF32>(mX, mW, p, clk, fz, st);
+    if (p.E <= 32) return launch_router_tc_t<1, WF32>(mX, mW, p, clk, fz, pdl, st);
+    if (p.E <= 64) return launch_router_tc_t<2, WF32>(mX, mW, p, clk, fz, pdl, st);
+    if (p.E <= 128) return launch_router_tc_t<4, WF32>(mX, mW, p, clk, fz, pdl, st);
+    return launch_router_tc_t<8, WF32>(mX, mW, p, clk, fz, pdl, st);
 }
 
 template <int KIND>
@@ -358,6 +374,8 @@ int launch_gemm(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap 
     return launch_status();
 }
 
+// A non-cooperative launch uses programmatic stream serialization: the kernel
+// waits for its predecessor before touching global memory.
 template <int KIND>
 int launch_decode(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &a2,
                   const CUtensorMap &a3, const CUtensorMap &a4, const DecArgs &args, int grid,
@@ -367,13 +385,14 @@ int launch_decode(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMa
     cfg.blockDim = dim3(DEC_THREADS, 1, 1);
     cfg.dynamicSmemBytes = DEC_SMEM_BYTES;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeCooperative;
     attr[0].val.cooperative = cooperative ? 1 : 0;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, grouped_gemm_decode_kernel<KIND>, a0, a1, a2, a3, a4, args) !=
-        cudaSuccess)
+    cfg.numAttrs = cooperative ? 1 : 2;
+    if (launch_ex(cfg, grouped_gemm_decode_kernel<KIND>, a0, a1, a2, a3, a4, args) != cudaSuccess)
         return MOE_ERR_CUDA;
     return launch_status();
 }
@@ -460,8 +479,8 @@ int router_impl(const void *x, int x_dtype, const void *W_g, int wg_dtype, const
             p.wg_parts = wg_parts_ws;
         }
         const RtcFuse &f = fuse ? *fz : off;
-        return wg_dtype == MOE_BF16 ? launch_router_tc<false>(p, dev->sms, f, st)
-                                    : launch_router_tc<true>(p, dev->sms, f, st);
+        return wg_dtype == MOE_BF16 ? launch_router_tc<false>(p, dev->sms, f, fuse, st)
+                                    : launch_router_tc<true>(p, dev->sms, f, fuse, st);
     }
     if (x_dtype == MOE_F32 && wg_dtype == MOE_F32) return launch_router_x<float, float>(p, st);
     if (x_dtype == MOE_BF16 && wg_dtype == MOE_F32) return launch_router_x<__nv_bfloat16, float>(p, st);

@@ -170,6 +170,10 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
         tma_prefetch_desc(&mX);
         if (!WF32 || presplit) tma_prefetch_desc(&mW);
     }
+    // Nothing above reads or writes global memory or TMEM, so it may overlap the
+    // previous kernel of the stream (programmatic launch); everything below follows it.
+    grid_dep_wait();
+    grid_dep_launch_dependents();
     if (warp == 1) {
         tmem_alloc(tmem_slot, tmem_cols);
         tmem_relinquish();
