@@ -10,8 +10,8 @@
 // global store is a 16-byte piece of a token's row.
 //
 // Same warp roles and pipeline as the prefill kernels (warp 0 TMA, warp 1 MMA,
-// warps 2-5 epilogue; an 8-stage ring of 16 KiB weights + 4 KiB tokens; two
-// 32-column accumulators).  Same arithmetic ("GLM-4.5 MoE Forward", How it works):
+// warps 2-5 epilogue; a ring of 10 (gate_up) or 8 (down) stages of 16 KiB weights
+// + 4 KiB tokens; two 32-column accumulators).  Same arithmetic ("GLM-4.5 MoE Forward", How it works):
 //
 // gate_up: one tile = 64 intermediate features of one expert x 32 tokens; A stacks
 //   the 64 gate rows and the matching 64 up rows, so TMEM lanes 0..63 hold the
@@ -32,7 +32,6 @@ namespace moe {
 constexpr int DEC_BM = 128;     // weight rows per tile (MMA M)
 constexpr int DEC_TT = 32;      // tokens per tile (MMA N)
 constexpr int DEC_BK = 64;
-constexpr int DEC_STAGES = 8;
 constexpr int DEC_THREADS = 192;
 constexpr int DEC_A_BYTES = DEC_BM * DEC_BK * 2;  // 16 KiB
 constexpr int DEC_B_BYTES = DEC_TT * DEC_BK * 2;  // 4 KiB
@@ -40,8 +39,21 @@ constexpr int DEC_STAGE_BYTES = DEC_A_BYTES + DEC_B_BYTES;
 constexpr int DEC_TMEM_COLS = 64;                 // 2 accumulators x 32 columns
 constexpr int DEC_EPI_LD = 132;                   // floats per token row of the transpose buffer
 constexpr int DEC_EPI_BYTES = DEC_TT * DEC_EPI_LD * 4;
-constexpr int DEC_SMEM_BYTES = 1024 + DEC_STAGES * DEC_STAGE_BYTES + 256 +
-                               (2 * GEMM_MAXE + 1) * 4 + DEC_EPI_BYTES + 64;
+// Ring depth per kernel.  A streaming kernel's bandwidth per SM is its bytes in
+// flight over the memory latency: gate_up takes 10 stages (200 KiB of weights in
+// flight; 2 % faster than 8 on the decode workloads).  The down kernel stays at 8:
+// its combine reads the slot partials through L1, which the larger shared-memory
+// carve-out shrinks (1-2 % slower at 10 stages).
+template <int KIND> __host__ __device__ constexpr int dec_stages() { return KIND == GEMM_GATE_UP ? 10 : 8; }
+template <int KIND> __host__ __device__ constexpr int dec_smem_bytes() {
+    return 1024 + dec_stages<KIND>() * DEC_STAGE_BYTES + 256 + (2 * GEMM_MAXE + 1) * 4 +
+           DEC_EPI_BYTES + 64;
+}
+static_assert(dec_smem_bytes<GEMM_GATE_UP>() <= 232448, "shared memory");
+static_assert(dec_smem_bytes<GEMM_DOWN>() <= 232448, "shared memory");
+// mbarriers (full/empty per stage, 2 tfull, 2 tempty, drain) and three words fit the
+// 256 bytes after the ring
+static_assert((2 * 10 + 5) * 8 + 12 <= 256, "barrier block");
 
 struct DecArgs {
     const int32_t *tile_off; // [E+1] prefix of 32-token tiles per expert
@@ -115,6 +127,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
                                const __grid_constant__ CUtensorMap mA_s0,
                                const __grid_constant__ CUtensorMap mA_s1,
                                const __grid_constant__ CUtensorMap mB_s, const DecArgs a) {
+    constexpr int DEC_STAGES = dec_stages<KIND>();
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));

@@ -383,7 +383,7 @@ int launch_decode(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMa
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid, 1, 1);
     cfg.blockDim = dim3(DEC_THREADS, 1, 1);
-    cfg.dynamicSmemBytes = DEC_SMEM_BYTES;
+    cfg.dynamicSmemBytes = dec_smem_bytes<KIND>();
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeCooperative;
@@ -402,10 +402,10 @@ int ensure_decode_attrs(DeviceInfo *dev) {
     if (dev->dec_attr_set) return MOE_OK;
     if (cudaFuncSetAttribute(grouped_gemm_decode_kernel<GEMM_GATE_UP>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             DEC_SMEM_BYTES) != cudaSuccess ||
+                             dec_smem_bytes<GEMM_GATE_UP>()) != cudaSuccess ||
         cudaFuncSetAttribute(grouped_gemm_decode_kernel<GEMM_DOWN>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             DEC_SMEM_BYTES) != cudaSuccess)
+                             dec_smem_bytes<GEMM_DOWN>()) != cudaSuccess)
         return MOE_ERR_CUDA;
     dev->dec_attr_set = true;
     return MOE_OK;
