@@ -21,6 +21,14 @@
  *   - Calls on one device may overlap only if they are on one stream: the
  *     kernels share nothing across calls except the status word, but two
  *     moe_forward calls must not share a workspace while both are in flight.
+ *   - Stream order is kept.  Some kernels use programmatic dependent launch
+ *     (the tensor-core router, the decode gate_up kernel).  They may be resident
+ *     before the previous work on the stream ends, but they touch no memory until
+ *     it has completed.  Kernels of this library also release their own
+ *     successors early (griddepcontrol.launch_dependents).  So a caller's kernel
+ *     launched right after with programmatic stream serialization must wait for
+ *     its predecessor (griddepcontrol.wait / cudaGridDependencySynchronize)
+ *     before it reads the outputs, as that launch mode requires anyway.
  */
 #ifndef MOE_B200_H
 #define MOE_B200_H
