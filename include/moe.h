@@ -92,6 +92,15 @@ int moe_router(const void *x, int x_dtype, const void *W_g, int wg_dtype, const 
 size_t moe_forward_workspace(int N, int D, int E, int d_moe, int d_sh, int k, int dtype);
 
 /*
+ * moe_layer_forward_workspace — bytes of workspace for moe_layer_forward's
+ * fastest path: moe_forward_workspace() plus, when wg_dtype is MOE_F32, room for
+ * the router matrix split into three bf16 parts (3 * E * D * 2 bytes).  0 for
+ * invalid sizes or dtypes.
+ */
+size_t moe_layer_forward_workspace(int N, int D, int E, int d_moe, int d_sh, int k, int dtype,
+                                   int wg_dtype);
+
+/*
  * moe_forward — routed experts, weighted combine and shared expert.
  * Defined by "GLM-4.5 MoE Forward", How it works: each routed expert is the
  * bias-free SwiGLU E_i(x) = W_down,i (SiLU(W_gate,i x) (.) W_up,i x) and
@@ -140,8 +149,11 @@ int moe_forward_clamped(const void *x, const void *gate_up, const void *down,
  * moe_layer_forward — the whole layer in one call: moe_router then moe_forward
  * ("GLM-4.5 Group Router" and "GLM-4.5 MoE Forward", How it works), with x's
  * dtype `dtype` for the tokens and the experts and wg_dtype for W_g.  Writes
- * topk_idx / topk_w (as moe_router) and y (as moe_forward); workspace as
- * moe_forward (moe_forward_workspace bytes).  For a bf16 layer of at most 128
+ * topk_idx / topk_w (as moe_router) and y (as moe_forward).  The workspace
+ * needs at least moe_forward_workspace() bytes; with
+ * moe_layer_forward_workspace() bytes (larger only for an fp32 W_g) a batch of
+ * several 128-token blocks splits W_g into bf16 parts once per call instead of
+ * once per token block (the same routing bit for bit, less router time).  For a bf16 layer of at most 128
  * tokens with at most 256 experts whose router runs on the tensor cores, the
  * forward's dispatch and token gather run inside the router kernel (one cluster
  * holds the whole routing), which saves two launches; the results are those of
@@ -189,7 +201,11 @@ int moe_bias_update(const int32_t *topk_idx, int N, int k, int E, float rate, fl
  *     N*k + 127*E up to a few thousand rows at D of a few hundred, fit).
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current.  Make it before any
- *     stream capture.
+ *     stream capture.  The address is cached per device and never looked up
+ *     again: after a cudaDeviceReset in the same process it is stale, so do
+ *     not use this entry point on a device reset after its first call.
+ *   - Arguments (sizes, dtype, pointers, an sm_100 device) are checked before
+ *     that look-up; errors as moe_forward.
  *   - All calls on a device share the array, which keeps the last call's
  *     contents.  Each call rewrites everything it reads before reading it.
  *     Calls whose kernels overlap on the GPU race; serialise them (one stream).
@@ -225,6 +241,17 @@ int moe_version(void);
  */
 int moe_debug_set_wait_limit_ns(uint64_t ns);
 int moe_debug_never_signal(int on);
+
+/*
+ * Test hook for the router's precision ("GLM-4.5 Group Router", How it works:
+ * the gate runs in float32).  While buf is non-null, every router launch
+ * (moe_router, moe_layer_forward) also writes each token's selection scores
+ * s' = sigmoid(r) + b as fp32 into buf [N, E] (device memory, 16-byte aligned,
+ * caller-owned, n_floats >= N * E, else the router call returns MOE_ERR_ARG
+ * before any launch).  The scores are those the selection compares, before
+ * any group masking.  buf = NULL turns the capture off (the default).
+ */
+int moe_debug_capture_scores(float *buf, size_t n_floats);
 
 /*
  * Profiling hooks (used by the benchmark; no effect on results).

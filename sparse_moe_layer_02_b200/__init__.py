@@ -18,9 +18,10 @@ import threading
 import torch
 
 __all__ = ["MoEError", "moe_router", "moe_forward", "moe_forward_workspace", "moe_layer",
+           "moe_layer_forward_workspace",
            "moe_device_status", "moe_status_string", "moe_debug_set_wait_limit_ns",
-           "moe_debug_never_signal", "moe_profile_set_events", "moe_launch_count",
-           "moe_forward_noalloc", "library_path", "load_library", "MOE_F32", "MOE_BF16",
+           "moe_debug_never_signal", "moe_debug_capture_scores", "moe_profile_set_events",
+           "moe_launch_count", "moe_forward_noalloc", "library_path", "load_library", "MOE_F32", "MOE_BF16",
            "EXPORTED_SYMBOLS", "moe_ep_symmetric_bytes", "moe_ep_workspace_bytes",
            "moe_ep_forward", "moe_ep_plan_host", "moe_ep_ipc_export", "moe_ep_ipc_open",
            "moe_ep_ipc_close", "ExpertParallelGroup", "MOE_EP_COUNT", "MOE_EP_SEND",
@@ -38,10 +39,11 @@ MOE_EP_ALL = 15
 MOE_EP_PHASES = (MOE_EP_COUNT, MOE_EP_SEND, MOE_EP_EXPERTS, MOE_EP_COMBINE)
 MOE_EP_IPC_HANDLE_BYTES = 72
 
-EXPORTED_SYMBOLS = ("moe_router", "moe_forward_workspace", "moe_forward", "moe_device_status",
+EXPORTED_SYMBOLS = ("moe_router", "moe_forward_workspace", "moe_layer_forward_workspace",
+                    "moe_forward", "moe_device_status",
                     "moe_status_string", "moe_version", "moe_debug_set_wait_limit_ns",
                     "moe_debug_never_signal", "moe_profile_set_events", "moe_launch_count",
-                    "moe_forward_noalloc", "moe_forward_clamped", "moe_layer_forward",
+                    "moe_debug_capture_scores", "moe_forward_noalloc", "moe_forward_clamped", "moe_layer_forward",
                     "moe_bias_update",
                     "moe_ep_symmetric_bytes",
                     "moe_ep_workspace_bytes", "moe_ep_forward", "moe_ep_plan_host",
@@ -73,6 +75,8 @@ def load_library():
         lib.moe_router.restype = I
         lib.moe_forward_workspace.argtypes = [I, I, I, I, I, I, I]
         lib.moe_forward_workspace.restype = ctypes.c_size_t
+        lib.moe_layer_forward_workspace.argtypes = [I, I, I, I, I, I, I, I]
+        lib.moe_layer_forward_workspace.restype = ctypes.c_size_t
         lib.moe_forward.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, P, P,
                                     ctypes.c_size_t, P]
         lib.moe_forward.restype = I
@@ -86,6 +90,8 @@ def load_library():
         lib.moe_debug_set_wait_limit_ns.restype = I
         lib.moe_debug_never_signal.argtypes = [I]
         lib.moe_debug_never_signal.restype = I
+        lib.moe_debug_capture_scores.argtypes = [P, ctypes.c_size_t]
+        lib.moe_debug_capture_scores.restype = I
         lib.moe_profile_set_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), I]
         lib.moe_profile_set_events.restype = I
         lib.moe_launch_count.argtypes = []
@@ -183,6 +189,15 @@ def moe_forward_workspace(N: int, D: int, E: int, d_moe: int, d_sh: int, k: int,
                                                      MOE_BF16 if dtype == torch.bfloat16 else MOE_F32))
 
 
+def moe_layer_forward_workspace(N: int, D: int, E: int, d_moe: int, d_sh: int, k: int,
+                                dtype: torch.dtype, wg_dtype: torch.dtype) -> int:
+    """Workspace bytes for moe_layer: moe_forward's plus, for an fp32 router matrix,
+    room to split it into bf16 parts once per call."""
+    f = lambda t: MOE_BF16 if t == torch.bfloat16 else MOE_F32
+    return int(load_library().moe_layer_forward_workspace(N, D, E, d_moe, d_sh, k, f(dtype),
+                                                           f(wg_dtype)))
+
+
 def moe_forward(x, gate_up, down, sh_gate, sh_up, sh_down, topk_idx, topk_w, y=None,
                 workspace=None, stream=None, gate_max=None, up_max=None):
     """Routed experts + weighted combine + shared expert; returns y [N, D].
@@ -260,7 +275,8 @@ def moe_layer(x, W_g, b, gate_up, down, sh_gate, sh_up, sh_down, n_group, topk_g
     if y is None:
         y = torch.empty((N, D), dtype=x.dtype, device=dev)
     if workspace is None:
-        workspace = torch.empty(max(moe_forward_workspace(N, D, E, d, d_sh, k, x.dtype), 256),
+        workspace = torch.empty(max(moe_layer_forward_workspace(N, D, E, d, d_sh, k, x.dtype,
+                                                                W_g.dtype), 256),
                                 dtype=torch.uint8, device=dev)
     if N == 0:
         return y, topk_idx, topk_w
@@ -303,6 +319,19 @@ def moe_debug_set_wait_limit_ns(ns: int):
 
 def moe_debug_never_signal(on: bool):
     _check(load_library().moe_debug_never_signal(int(bool(on))), "moe_debug_never_signal")
+
+
+def moe_debug_capture_scores(buf) -> None:
+    """Test hook: while `buf` (a contiguous fp32 CUDA tensor of at least N*E
+    elements) is set, router launches also write their selection scores
+    s' = sigmoid(r) + b into it as [N, E]; None turns the capture off."""
+    if buf is None:
+        _check(load_library().moe_debug_capture_scores(None, 0), "moe_debug_capture_scores")
+        return
+    if buf.dtype != torch.float32:
+        raise ValueError("the score buffer must be float32")
+    _check(load_library().moe_debug_capture_scores(_dev(buf, "buf"), buf.numel()),
+           "moe_debug_capture_scores")
 
 
 def moe_profile_set_events(events) -> None:

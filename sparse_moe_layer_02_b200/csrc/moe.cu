@@ -26,6 +26,9 @@ constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;
 constexpr int kDecodeMaxTokens = 256;
 uint64_t g_wait_limit_ns = kDefaultWaitLimitNs;
 int g_never_signal = 0;
+// Test hook: device buffer receiving the router's selection scores s' (null: off).
+float *g_dbg_sp = nullptr;
+size_t g_dbg_sp_n = 0;
 
 std::atomic<unsigned long long> g_launches{0};
 constexpr int kMaxProfEvents = 16;
@@ -107,14 +110,17 @@ int check_router_shape(int N, int D, int E, int G, int tg, int k) {
 // ---------------------------------------------------------------------------
 struct WsLayout {
     size_t chunk_hist, counts, tile_off, meta, pos_of, perm_tok, w_perm;
-    size_t x_perm, h_perm, h_sh, slot, osh, wg_parts, total;
+    size_t x_perm, h_perm, h_sh, slot, osh, wg_parts, total, total_with_parts;
     int nchunks;
     size_t rows_max;
     bool decode;
     int tile_rows;
 };
 
-bool plan_workspace(int N, int D, int E, int d, int d_sh, int k, int dtype, WsLayout &L) {
+// with_wg_parts: also reserve the three bf16 parts of an fp32 router matrix
+// (moe_layer_forward's split-once path); moe_forward never uses them.
+bool plan_workspace(int N, int D, int E, int d, int d_sh, int k, int dtype, WsLayout &L,
+                    bool with_wg_parts = false) {
     if (N < 0 || D <= 0 || E <= 0 || d <= 0 || d_sh <= 0 || k <= 0) return false;
     if (dtype != MOE_F32 && dtype != MOE_BF16) return false;
     const size_t es = dtype == MOE_BF16 ? 2 : 4;
@@ -146,9 +152,10 @@ bool plan_workspace(int N, int D, int E, int d, int d_sh, int k, int dtype, WsLa
     L.slot = take(L.rows_max * D * es);
     // fp32 output of the shared expert, combined with the slots (prefill kernels)
     L.osh = take(dtype == MOE_BF16 && !L.decode ? (size_t)N * D * 4 : 0);
-    // the router matrix split into three bf16 parts (moe_layer_forward, fp32 W_g)
-    L.wg_parts = take((size_t)3 * E * D * 2);
     L.total = off;
+    // the router matrix split into three bf16 parts (moe_layer_forward, fp32 W_g)
+    L.wg_parts = take(with_wg_parts ? (size_t)3 * E * D * 2 : 0);
+    L.total_with_parts = off;
     return true;
 }
 
@@ -462,6 +469,11 @@ int router_impl(const void *x, int x_dtype, const void *W_g, int wg_dtype, const
     p.topk_idx = topk_idx;
     p.topk_w = topk_w;
     p.wg_parts = nullptr;
+    p.dbg_sp = nullptr;
+    if (g_dbg_sp) {
+        if (g_dbg_sp_n < (size_t)N * E) return MOE_ERR_ARG;
+        p.dbg_sp = g_dbg_sp;
+    }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     RtcFuse off = {};
     const bool tc = x_dtype == MOE_BF16 && E % 16 == 0 && E >= 16 && D % 8 == 0 &&
@@ -523,6 +535,13 @@ int moe_debug_never_signal(int on) {
     return MOE_OK;
 }
 
+int moe_debug_capture_scores(float *buf, size_t n_floats) {
+    if (buf && (!aligned16(buf) || n_floats == 0)) return MOE_ERR_ARG;
+    g_dbg_sp = buf;
+    g_dbg_sp_n = buf ? n_floats : 0;
+    return MOE_OK;
+}
+
 int moe_profile_set_events(void *const *events, int n) {
     if (n < 0 || n > kMaxProfEvents || (n > 0 && !events)) return MOE_ERR_ARG;
     for (int i = 0; i < n; ++i) g_prof_events[i] = events[i];
@@ -558,6 +577,14 @@ size_t moe_forward_workspace(int N, int D, int E, int d_moe, int d_sh, int k, in
     WsLayout L;
     if (!plan_workspace(N, D, E, d_moe, d_sh, k, dtype, L)) return 0;
     return L.total;
+}
+
+size_t moe_layer_forward_workspace(int N, int D, int E, int d_moe, int d_sh, int k, int dtype,
+                                   int wg_dtype) {
+    if (wg_dtype != MOE_F32 && wg_dtype != MOE_BF16) return 0;
+    WsLayout L;
+    if (!plan_workspace(N, D, E, d_moe, d_sh, k, dtype, L, wg_dtype == MOE_F32)) return 0;
+    return L.total_with_parts;
 }
 
 }  // extern "C"
@@ -879,6 +906,14 @@ int moe_layer_forward(const void *x, const void *W_g, int wg_dtype, const float 
                             d_moe, d_sh, k, dtype, y, workspace, ws_bytes, L)) != MOE_OK)
         return rc;
     if (N == 0) return MOE_OK;
+    // The split-once scratch for an fp32 W_g is used when the workspace covers it
+    // (moe_layer_forward_workspace); with moe_forward_workspace bytes the router
+    // splits W_g in every token block instead (the same routing, bit for bit).
+    WsLayout Lp;
+    plan_workspace(N, D, E, d_moe, d_sh, k, dtype, Lp, wg_dtype == MOE_F32);
+    void *wg_parts_ws = wg_dtype == MOE_F32 && ws_bytes >= Lp.total_with_parts
+                            ? static_cast<void *>(static_cast<uint8_t *>(workspace) + Lp.wg_parts)
+                            : nullptr;
     if (!W_g || !b || !aligned16(W_g) || !aligned16(b)) return MOE_ERR_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
@@ -894,7 +929,7 @@ int moe_layer_forward(const void *x, const void *W_g, int wg_dtype, const float 
     }
     bool fused = false;
     rc = router_impl(x, dtype, W_g, wg_dtype, b, N, D, E, n_group, topk_group, k, norm_topk_prob,
-                     alpha, topk_idx, topk_w, stream, &fz, &fused, ws + L.wg_parts);
+                     alpha, topk_idx, topk_w, stream, &fz, &fused, wg_parts_ws);
     if (rc != MOE_OK) return rc;
     prof.mark();
     return forward_impl(x, gate_up, down, sh_gate, sh_up, sh_down, topk_idx, topk_w, N, D, E, d_moe,

@@ -14,7 +14,9 @@
 // of the array is only a stand-in, not a device address, so it is never passed
 // to a kernel.  The address is cached per device.  Make the first call on a
 // device before any stream capture, since the set-up call is not a stream
-// operation.
+// operation.  The cache is never refreshed: after cudaDeviceReset in the same
+// process the cached address is stale, so this entry point must not be used on
+// a device that was reset after its first call.
 //
 // Sharing: every call on a device uses the same array and the array keeps the
 // last call's contents.  Everything the kernels need zeroed or initialised per
@@ -37,19 +39,35 @@ void *g_scratch_addr[kMaxScratchDevices];
 std::mutex g_scratch_mu;
 
 // Device address of the scratch array on the current device (looked up once).
+// Only an sm_100 device can load this library's kernels, so any other device is
+// refused before the lookup, which would otherwise try to load the module there.
 int scratch_on_current_device(void **out) {
     int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxScratchDevices)
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxScratchDevices) {
+        cudaGetLastError();
         return MOE_ERR_CUDA;
+    }
+    int major = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) {
+        cudaGetLastError();
+        return MOE_ERR_CUDA;
+    }
+    if (major != 10) return MOE_ERR_NO_DEVICE;
     std::lock_guard<std::mutex> lk(g_scratch_mu);
     if (!g_scratch_addr[dev]) {
         void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return MOE_ERR_CUDA;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+            // leave no sticky error behind for the next call's launch check
+            cudaGetLastError();
+            return MOE_ERR_CUDA;
+        }
         g_scratch_addr[dev] = p;
     }
     *out = g_scratch_addr[dev];
     return MOE_OK;
 }
+
+bool ok_ptr(const void *p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 }  // namespace
 
@@ -65,6 +83,10 @@ extern "C" int moe_forward_noalloc(const void *x, const void *gate_up, const voi
     // before any launch, with the workspace error code.
     if (need > MOE_NOALLOC_SCRATCH_BYTES) return MOE_ERR_WORKSPACE;
     if (N == 0) return MOE_OK;
+    // The caller's pointers are checked before the set-up below touches the device.
+    const void *ptrs[] = {x, gate_up, down, sh_gate, sh_up, sh_down, topk_idx, topk_w, y};
+    for (const void *q : ptrs)
+        if (!ok_ptr(q)) return MOE_ERR_ARG;
     void *scratch = nullptr;
     const int rc = scratch_on_current_device(&scratch);
     if (rc != MOE_OK) return rc;

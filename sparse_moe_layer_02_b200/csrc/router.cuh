@@ -38,6 +38,9 @@ struct RouterParams {
     // fp32 W_g already split into three bf16 parts [3][E][D] (null: the tensor-core
     // router splits it itself, per token block)
     const void *wg_parts;
+    // Test hook (null on the hot path): receives every token's fp32 selection
+    // scores s' = sigmoid(r) + b [N][E], before any group masking.
+    float *dbg_sp;
 };
 
 // Dynamic shared memory of router_kernel<EV>: x chunk, W chunk, partial logits,
@@ -84,6 +87,7 @@ __device__ __forceinline__ void router_select(const RouterParams &p, int t, cons
         if (e < E) {
             s[v] = 1.0f / (1.0f + expf(-logit[v]));
             sp[v] = s[v] + p.b[e];
+            if (p.dbg_sp) p.dbg_sp[(size_t)t * E + e] = sp[v];
         }
     }
     // Candidate mask over this lane's experts (bit v).

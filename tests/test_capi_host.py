@@ -92,6 +92,20 @@ def test_workspace_sizes():
     assert big < 6 * 2 ** 30
 
 
+def test_layer_workspace_adds_router_parts_for_fp32_matrix_only():
+    lib = moe.load_library()
+    fw = lambda *a: lib.moe_forward_workspace(*a)
+    lw = lambda *a: lib.moe_layer_forward_workspace(*a)
+    for N, D, E in [(8192, 5120, 160), (300, 520, 48), (32, 4096, 128)]:
+        base = fw(N, D, E, 256, 256, 8, 1)
+        # fp32 W_g: three bf16 parts of E x D, 256-byte aligned
+        parts = (3 * E * D * 2 + 255) // 256 * 256
+        assert lw(N, D, E, 256, 256, 8, 1, 0) == base + parts
+        assert lw(N, D, E, 256, 256, 8, 1, 1) == base       # bf16 W_g: no split
+    assert lw(10, 64, 16, 32, 32, 2, 1, 7) == 0            # bad router dtype
+    assert lw(10, 64, 16, 32, 32, 2, 9, 0) == 0            # bad dtype
+
+
 def test_layer_call_rejects_bad_arguments_before_any_launch():
     lib = moe.load_library()
     call = lambda **kw: lib.moe_layer_forward(

@@ -93,7 +93,8 @@ def test_ep_emulated_equals_single_device(P, Ns):
     y_orc = oracle.forward(host(xs[0]), host(inp.gate_up), host(inp.down), host(inp.sh_gate),
                            host(inp.sh_up), host(inp.sh_down), host(ids[0]).numpy(),
                            host(wts[0]).double().numpy())
-    assert rel_err(ys[0].float().cpu().numpy(), y_orc)["max_rel"] <= Y_TOL[torch.bfloat16]
+    e = rel_err(ys[0].float().cpu().numpy(), y_orc)
+    assert e["max_rel"] <= Y_TOL[torch.bfloat16] and e["max_row_l2_rel"] <= Y_TOL[torch.bfloat16]
 
 
 def test_ep_emulated_small_batches():
@@ -109,6 +110,7 @@ def test_ep_emulated_small_batches():
                                 inp.sh_down, ids[r], wts[r])
         err = rel_err(ys[r].float().cpu().numpy(), y_ref.float().cpu().numpy())
         assert err["max_rel"] <= Y_TOL[torch.bfloat16]
+        assert err["max_row_l2_rel"] <= Y_TOL[torch.bfloat16]
 
 
 def test_ep_missing_rank_times_out_and_context_survives():

@@ -22,7 +22,11 @@ from workloads import CONFIGS, make_inputs
 from _parity import Y_TOL, rel_err
 
 CASES = {
+    # more than 256 tokens: the 128-row tile kernels and the combine launch
     "bf16": CONFIGS["glm5_prefill"].with_(N=300, D=512, E=8, k=4, d_moe=256, d_sh=256),
+    # at most 256 tokens: the decode kernels, whose down kernel waits on a per-call
+    # tile counter in the scratch before it combines (the latency-bound callers)
+    "bf16_decode": CONFIGS["air_decode"].with_(N=64, D=1024, E=32, k=8, d_moe=512, d_sh=512),
     "fp32": CONFIGS["tiny_fp32"],
 }
 
@@ -54,6 +58,9 @@ def test_noalloc_matches_workspace_entry_point_twice(case):
         err = rel_err(y.float().cpu().numpy(), y_ref.float().cpu().numpy())
         assert err["finite"], "call %d left non-finite values" % call
         assert err["max_rel"] <= Y_TOL[cfg.dtype], (call, err)
+        # the same kernels on the same inputs: the forward is deterministic, so the
+        # outputs agree bit for bit
+        assert torch.equal(y, y_ref), (call, err)
 
 
 def test_noalloc_refuses_sizes_beyond_its_scratch():
@@ -64,3 +71,5 @@ def test_noalloc_refuses_sizes_beyond_its_scratch():
     rc = lib.moe_forward_noalloc(*([None] * 8), c.N, c.D, c.E, c.d_moe, c.d_sh, c.k, 1, None, None)
     assert rc == -4
     assert lib.moe_forward_noalloc(*([None] * 8), 10, 64, 8, 32, 32, 2, 9, None, None) == -3
+    # null pointers are refused before the scratch address is looked up on a device
+    assert lib.moe_forward_noalloc(*([None] * 8), 10, 64, 8, 32, 32, 2, 1, None, None) == -1
