@@ -72,6 +72,9 @@ def parse_args():
                     help="target duration of the oracle's CPU-baseline sample")
     ap.add_argument("--set", action="append", default=[], metavar="FIELD=VALUE",
                     help="override a size of the workload (e.g. E=32) for small profiling cases")
+    ap.add_argument("--pair", default="off", choices=["off", "on", "pad"],
+                    help="prefill expert GEMMs on CTA pairs: never (default), full pairs with "
+                         "one-SM tails, padded pairs only")
     ap.add_argument("--graph", action="store_true",
                     help="capture the K timed steps as one CUDA graph and time one replay "
                          "(default: launch them one by one)")
@@ -704,6 +707,7 @@ def main():
 
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=60), device_id=dev)
 
+    moe.moe_debug_set_pair_mode({"off": 0, "on": 1, "pad": 2}[args.pair])
     cfg, over = workload(args.workload, args.set)
     head = measure(cfg, over, args, dev, dist, rank, world, local, moe, full=True)
     cpu, par = None, None
@@ -739,6 +743,7 @@ def main():
         "e2e": head["e2e"],
         "gpu_launches": head["gpu_launches"],
         "timing": head["timing"],
+        "gemm_pairs": args.pair,
         "clocks": head["clocks"],
         "workloads": {
             name: {"value": res["value"], "unit": UNIT, "ms_per_step": res["ms_per_step"],

@@ -243,6 +243,18 @@ int moe_debug_set_wait_limit_ns(uint64_t ns);
 int moe_debug_never_signal(int on);
 
 /*
+ * Tuning and test hook for the prefill expert GEMMs (more than 256 bf16
+ * tokens).  Mode 1 runs them on CTA pairs (two SMs share one M = 256
+ * tensor-core tile) with the odd last m-tile of each expert on the one-SM
+ * kernels; mode 2 runs every m-tile on CTA pairs, an odd last m-tile pairing
+ * with an empty half; modes 0 and -1 (the default) run every tile on the
+ * one-SM kernels, which were the faster ones on every configuration measured.
+ * Results are identical bit for bit in every mode.  MOE_ERR_ARG for other
+ * values.
+ */
+int moe_debug_set_pair_mode(int mode);
+
+/*
  * Test hook for the router's precision ("GLM-4.5 Group Router", How it works:
  * the gate runs in float32).  While buf is non-null, every router launch
  * (moe_router, moe_layer_forward) also writes each token's selection scores

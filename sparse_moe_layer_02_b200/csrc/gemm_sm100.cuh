@@ -49,11 +49,12 @@ constexpr int GEMM_MAXE = 512;
 constexpr int GEMM_OUT_BOX = 32;                                   // rows and columns of a store box
 constexpr int GEMM_OUT_BUF = GEMM_OUT_BOX * GEMM_OUT_BOX * 2;     // 2 KiB
 constexpr int GEMM_STG_OFF =
-    (GEMM_STAGES * GEMM_STAGE_BYTES + 256 + (GEMM_MAXE + 1) * 4 + 1023) / 1024 * 1024;
+    (GEMM_STAGES * GEMM_STAGE_BYTES + 256 + 2 * (GEMM_MAXE + 1) * 4 + 1023) / 1024 * 1024;
 constexpr int GEMM_SMEM_BYTES = 1024 + GEMM_STG_OFF + 4 * 2 * GEMM_OUT_BUF;
 static_assert(GEMM_SMEM_BYTES <= 232448, "shared memory");
 
 enum GemmKind { GEMM_GATE_UP = 0, GEMM_DOWN = 1 };
+enum GemmTiles { GEMM_ALL_TILES = 0, GEMM_TAIL_TILES = 1, GEMM_PAIR_PAD = 2 };
 
 constexpr int EP_MAX_RANKS = 8; // ranks of an expert-parallel group
 
@@ -98,6 +99,10 @@ struct GemmArgs {
     int never_signal;
     float gate_max, up_max; // gate_up: SwiGLU limits (+infinity = plain SwiGLU)
     int tma_out;            // down: routed rows stored by TMA through the mOut map
+    // Tiles taken by the one-CTA kernel: GEMM_ALL_TILES, or GEMM_TAIL_TILES = only
+    // the last m-tile of every expert with an odd m-tile count (and the last shared
+    // m-tile when their count is odd), the tiles the CTA-pair kernel leaves over.
+    int mode;
     // Expert parallelism (all null / 0 for a single-device layer).  The routed
     // rows are other ranks' tokens received into this rank's buffer.
     const uint32_t *ep_wait_ctr;    // gate_up: rows arrived (this epoch) ...
@@ -109,6 +114,7 @@ struct GemmArgs {
 };
 
 struct TileCoord {
+    bool valid; // false: the odd half of a padded pair tile (no rows; nothing loaded or stored)
     bool shared;
     int e;     // routed expert
     int a_row; // row coordinate in the A map
@@ -116,31 +122,82 @@ struct TileCoord {
     int kb;    // k-blocks
 };
 
+// Exclusive prefix over the experts (one warp): out[e] = sum_{j < e} f(j) for
+// e in [0, E], with f(j) from expert j's m-tile count m (tile prefix tile_off):
+// kind 0 the full pairs m / 2, kind 1 the odd tail m % 2, kind 2 the pairs
+// including a half-empty last one, (m + 1) / 2.
+__device__ __forceinline__ void warp_expert_prefix(const int *tile_off, int E, int *out, int kind,
+                                                   int lane) {
+    int carry = 0;
+    for (int base = 0; base <= E; base += 32) {
+        const int e = base + lane;
+        int v = 0;
+        if (e < E) {
+            const int m = tile_off[e + 1] - tile_off[e];
+            v = kind == 1 ? (m & 1) : kind == 2 ? ((m + 1) >> 1) : (m >> 1);
+        }
+        int incl = v;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int n = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += n;
+        }
+        if (e <= E) out[e] = carry + incl - v;
+        carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+}
+
+// Largest e in [0, E) with pre[e] * nb <= t (pre non-decreasing, pre[0] = 0).
+__device__ __forceinline__ int find_expert(const int *pre, int E, int nb, int t) {
+    int lo = 0, hi = E - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (pre[mid] * nb <= t) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+// s_aux: the tail prefix (warp_expert_prefix with odd = 1) in GEMM_TAIL_TILES mode.
 __device__ __forceinline__ TileCoord decode_tile(int t, int routed_tiles, const GemmArgs &a,
-                                                 const int *s_tile_off) {
+                                                 const int *s_tile_off, const int *s_aux) {
     TileCoord c;
     if (t < routed_tiles) {
+        if (a.mode == GEMM_TAIL_TILES) {
+            // one odd tail m-tile per listed expert, its n-blocks consecutive
+            const int e = find_expert(s_aux, a.E, a.nb_r, t);
+            c.nb = t - s_aux[e] * a.nb_r;
+            c.valid = true;
+            c.shared = false;
+            c.e = e;
+            c.a_row = (s_tile_off[e + 1] - 1) * GEMM_BM;
+            c.kb = a.kb_r;
+            return c;
+        }
         // Expert-major order: expert e owns tiles [tile_off[e] * nb_r, tile_off[e+1] * nb_r),
         // n-block-major inside, so the m-tiles that read the same weight tile are
         // neighbours in the round-robin and run at the same time (one HBM read,
         // the others hit L2).
-        int lo = 0, hi = a.E - 1;
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (s_tile_off[mid] * a.nb_r <= t) lo = mid; else hi = mid - 1;
-        }
+        const int lo = find_expert(s_tile_off, a.E, a.nb_r, t);
         const int mte = s_tile_off[lo + 1] - s_tile_off[lo];
         const int local = t - s_tile_off[lo] * a.nb_r;
         c.nb = local / mte;
         const int mt = s_tile_off[lo] + (local - c.nb * mte);
+        c.valid = true;
         c.shared = false;
         c.e = lo;
         c.a_row = mt * GEMM_BM;
         c.kb = a.kb_r;
     } else {
         const int t2 = t - routed_tiles;
-        const int mt = t2 / a.nb_s;
-        c.nb = t2 - mt * a.nb_s;
+        int mt;
+        if (a.mode == GEMM_TAIL_TILES) {
+            mt = a.mt_s - 1;
+            c.nb = t2;
+        } else {
+            mt = t2 / a.nb_s;
+            c.nb = t2 - mt * a.nb_s;
+        }
+        c.valid = true;
         c.shared = true;
         c.e = -1;
         c.a_row = mt * GEMM_BM;
@@ -271,6 +328,134 @@ __global__ void __launch_bounds__(COMBINE_THREADS, 2) combine_kernel(const GemmA
     combine_rows(g, blockIdx.x * W + (threadIdx.x >> 5), gridDim.x * W, threadIdx.x & 31);
 }
 
+// Epilogue of one tile for the 32 rows of TMEM lane quadrant q (thread `lane`
+// owns row q * 32 + lane of the tile): gate_up writes h = SwiGLU(gate, up) in
+// bf16; down writes the routed rows scaled by their routing weight (bf16 slot
+// partials, by TMA through mOut or per thread) or the shared expert's fp32 rows.
+// tbase: the accumulator's TMEM address at this warp's lane quadrant.  stg /
+// nstore: this warp's two store staging buffers and the boxes staged so far.
+template <int KIND>
+__device__ __forceinline__ void epilogue_tile(const GemmArgs &a, const CUtensorMap &mOut,
+                                              const TileCoord &c, uint32_t tbase, int q, int lane,
+                                              uint8_t *stg, uint32_t &nstore) {
+    const int row = q * 32 + lane;
+    if (KIND == GEMM_GATE_UP) {
+        __nv_bfloat16 *out = c.shared ? a.out_s : a.out_r;
+        const int ld = c.shared ? a.ld_s : a.ld_r;
+        const int ncols = c.shared ? a.ncols_s : a.ncols_r;
+        const int grow = c.a_row + row;
+        const bool row_ok = c.shared ? (grow < a.N) : true;
+        __nv_bfloat16 *row_ptr = out + (size_t)grow * ld;
+#pragma unroll 1
+        for (int ch = 0; ch < 4; ++ch) {
+            uint32_t g[32], u[32];
+            tmem_ld_32x32b_x32(tbase + ch * 32, g);
+            tmem_ld_32x32b_x32(tbase + 128 + ch * 32, u);
+            tmem_ld_wait();
+            const int col = c.nb * 128 + ch * 32;
+            if (row_ok && col < ncols) {
+                float h[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    h[i] = swiglu_f(__uint_as_float(g[i]), __uint_as_float(u[i]),
+                                    a.gate_max, a.up_max);
+                store_row_chunk_bf16(row_ptr, col, ncols, h);
+            }
+        }
+    } else if (!c.shared && a.tma_out) {
+        // Routed rows are contiguous in the slot buffer: each 32-column chunk
+        // of this warp's 32 rows is staged in shared memory and written by
+        // one TMA store (full lines, off the epilogue threads' critical path).
+        const float wr = a.w_perm[c.a_row + row];
+#pragma unroll 1
+        for (int ch = 0; ch < 8; ++ch) {
+            uint32_t v[32];
+            tmem_ld_32x32b_x32(tbase + ch * 32, v);
+            tmem_ld_wait();
+            const int col = c.nb * GEMM_BN + ch * 32;
+            if (col < a.ncols_r) {
+                uint8_t *buf = stg + (nstore & 1) * GEMM_OUT_BUF;
+                if (lane == 0) bulk_wait_group_read<1>(); // the box staged 2 ago left buf
+                __syncwarp();
+                uint32_t pk[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    pk[i] = pack_bf16x2(wr * __uint_as_float(v[2 * i]),
+                                        wr * __uint_as_float(v[2 * i + 1]));
+                const uint4 u[4] = {make_uint4(pk[0], pk[1], pk[2], pk[3]),
+                                    make_uint4(pk[4], pk[5], pk[6], pk[7]),
+                                    make_uint4(pk[8], pk[9], pk[10], pk[11]),
+                                    make_uint4(pk[12], pk[13], pk[14], pk[15])};
+                uint4 *dst = reinterpret_cast<uint4 *>(buf + lane * (GEMM_OUT_BOX * 2));
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    // rotate the pieces across lanes (fewer bank conflicts); the
+                    // selects keep the data in registers
+                    const int p = (j + lane) & 3;
+                    const uint4 val = p == 0 ? u[0] : p == 1 ? u[1] : p == 2 ? u[2] : u[3];
+                    dst[p] = val;
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(&mOut, buf, col, c.a_row + q * 32);
+                    bulk_commit_group();
+                }
+                ++nstore;
+            }
+        }
+    } else if (!c.shared) {
+        const int grow = c.a_row + row;
+        float wr;
+        __nv_bfloat16 *row_ptr;
+        int src = 0;
+        if (a.ep_P > 0) {
+            // the row goes back to its token's rank, at the token's pair id;
+            // padding rows carry source -1 and are not stored
+            const int4 m = a.ep_meta[grow];
+            src = (m.x >= 0 && m.x < a.ep_P) ? m.x : -1;
+            wr = __int_as_float(m.z);
+            row_ptr = src >= 0 ? a.ep_out[src] + (size_t)m.y * a.ld_r : nullptr;
+        } else {
+            wr = a.w_perm[grow];
+            row_ptr = a.out_r + (size_t)grow * a.ld_r;
+        }
+#pragma unroll 1
+        for (int ch = 0; ch < 8; ++ch) {
+            uint32_t v[32];
+            tmem_ld_32x32b_x32(tbase + ch * 32, v);
+            tmem_ld_wait();
+            const int col = c.nb * GEMM_BN + ch * 32;
+            if (row_ptr && col < a.ncols_r) {
+                float o[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) o[i] = wr * __uint_as_float(v[i]);
+                store_row_chunk_bf16(row_ptr, col, a.ncols_r, o);
+            }
+        }
+        if (a.ep_P > 0) warp_count_rows(a.ep_ret, src, a.ep_P);
+    } else {
+        // shared expert: fp32 output rows, added last by combine_kernel
+        const int n = c.a_row + row;
+        float *row_ptr = a.osh + (size_t)n * a.ld_s;
+#pragma unroll 1
+        for (int ch = 0; ch < 8; ++ch) {
+            uint32_t v[32];
+            tmem_ld_32x32b_x32(tbase + ch * 32, v);
+            tmem_ld_wait();
+            const int col = c.nb * GEMM_BN + ch * 32;
+            if (n < a.N && col < a.ncols_s) {
+#pragma unroll
+                for (int qv = 0; qv < 8; ++qv)
+                    if (col + 4 * qv < a.ncols_s)
+                        reinterpret_cast<float4 *>(row_ptr + col)[qv] =
+                            make_float4(__uint_as_float(v[4 * qv]), __uint_as_float(v[4 * qv + 1]),
+                                        __uint_as_float(v[4 * qv + 2]), __uint_as_float(v[4 * qv + 3]));
+            }
+        }
+    }
+}
+
 // mOut (down with tma_out): the slot rows [rows, D] bf16, box 32 x 32, no swizzle.
 template <int KIND>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
@@ -292,6 +477,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     int *s_tile_off = reinterpret_cast<int *>(smem + GEMM_STAGES * GEMM_STAGE_BYTES + 256);
+    int *s_aux = s_tile_off + (GEMM_MAXE + 1);
 
     const int warp = warp_id(), lane = lane_id();
 
@@ -324,6 +510,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    if (a.mode == GEMM_TAIL_TILES) {
+        if (warp == 2) warp_expert_prefix(s_tile_off, a.E, s_aux, 1, lane);
+        __syncthreads();
+    }
 
     const uint64_t limit = a.wait_limit_ns;
     if (a.ep_wait_ctr) {
@@ -344,8 +534,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         }
         __syncthreads();
     }
-    const int routed_tiles = a.meta[2] * a.nb_r;
-    const int total_tiles = *abort_flag ? 0 : routed_tiles + a.mt_s * a.nb_s;
+    const bool tails = a.mode == GEMM_TAIL_TILES;
+    const int routed_tiles = (tails ? s_aux[a.E] : a.meta[2]) * a.nb_r;
+    const int shared_tiles = tails ? ((a.mt_s & 1) ? a.nb_s : 0) : a.mt_s * a.nb_s;
+    const int total_tiles = *abort_flag ? 0 : routed_tiles + shared_tiles;
 
     if (warp == 0) {
         // ------------------------------ TMA producer ------------------------------
@@ -353,7 +545,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             uint32_t it = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
-                const TileCoord c = decode_tile(t, routed_tiles, a, s_tile_off);
+                const TileCoord c = decode_tile(t, routed_tiles, a, s_tile_off, s_aux);
                 const CUtensorMap *mA = c.shared ? &mA_s : &mA_r;
                 // Tiles of one n-block (same weight tile) start at the same k-block and
                 // share each weight line as it arrives; the n-blocks of one m-tile
@@ -403,7 +595,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             uint32_t it = 0, tc = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++tc) {
-                const TileCoord c = decode_tile(t, routed_tiles, a, s_tile_off);
+                const TileCoord c = decode_tile(t, routed_tiles, a, s_tile_off, s_aux);
                 const uint32_t acc = tc & 1, aph = (tc >> 1) & 1;
                 if (!mbar_wait(&tempty[acc], aph ^ 1, limit, abort_flag, 110)) { ok = false; break; }
                 tc_fence_after();
@@ -439,7 +631,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         uint32_t nstore = 0;             // store boxes this warp has staged
         uint32_t tc = 0;
         for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++tc) {
-            const TileCoord c = decode_tile(t, routed_tiles, a, s_tile_off);
+            const TileCoord c = decode_tile(t, routed_tiles, a, s_tile_off, s_aux);
             const uint32_t acc = tc & 1, aph = (tc >> 1) & 1;
             // After an abort every wait fails at once; the loop still walks the same
             // tiles in every epilogue warp so the named barriers stay matched.
@@ -453,121 +645,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             tc_fence_after();
             const uint32_t tbase = tmem_base + acc * GEMM_BN + ((uint32_t)(q * 32) << 16);
 
-            if (KIND == GEMM_GATE_UP) {
-                __nv_bfloat16 *out = c.shared ? a.out_s : a.out_r;
-                const int ld = c.shared ? a.ld_s : a.ld_r;
-                const int ncols = c.shared ? a.ncols_s : a.ncols_r;
-                const int grow = c.a_row + row;
-                const bool row_ok = c.shared ? (grow < a.N) : true;
-                __nv_bfloat16 *row_ptr = out + (size_t)grow * ld;
-#pragma unroll 1
-                for (int ch = 0; ch < 4; ++ch) {
-                    uint32_t g[32], u[32];
-                    tmem_ld_32x32b_x32(tbase + ch * 32, g);
-                    tmem_ld_32x32b_x32(tbase + 128 + ch * 32, u);
-                    tmem_ld_wait();
-                    const int col = c.nb * 128 + ch * 32;
-                    if (row_ok && col < ncols) {
-                        float h[32];
-#pragma unroll
-                        for (int i = 0; i < 32; ++i)
-                            h[i] = swiglu_f(__uint_as_float(g[i]), __uint_as_float(u[i]),
-                                            a.gate_max, a.up_max);
-                        store_row_chunk_bf16(row_ptr, col, ncols, h);
-                    }
-                }
-            } else if (!c.shared && a.tma_out) {
-                // Routed rows are contiguous in the slot buffer: each 32-column chunk
-                // of this warp's 32 rows is staged in shared memory and written by
-                // one TMA store (full lines, off the epilogue threads' critical path).
-                const float wr = a.w_perm[c.a_row + row];
-#pragma unroll 1
-                for (int ch = 0; ch < 8; ++ch) {
-                    uint32_t v[32];
-                    tmem_ld_32x32b_x32(tbase + ch * 32, v);
-                    tmem_ld_wait();
-                    const int col = c.nb * GEMM_BN + ch * 32;
-                    if (col < a.ncols_r) {
-                        uint8_t *buf = stg + (nstore & 1) * GEMM_OUT_BUF;
-                        if (lane == 0) bulk_wait_group_read<1>(); // the box staged 2 ago left buf
-                        __syncwarp();
-                        uint32_t pk[16];
-#pragma unroll
-                        for (int i = 0; i < 16; ++i)
-                            pk[i] = pack_bf16x2(wr * __uint_as_float(v[2 * i]),
-                                                wr * __uint_as_float(v[2 * i + 1]));
-                        const uint4 u[4] = {make_uint4(pk[0], pk[1], pk[2], pk[3]),
-                                            make_uint4(pk[4], pk[5], pk[6], pk[7]),
-                                            make_uint4(pk[8], pk[9], pk[10], pk[11]),
-                                            make_uint4(pk[12], pk[13], pk[14], pk[15])};
-                        uint4 *dst = reinterpret_cast<uint4 *>(buf + lane * (GEMM_OUT_BOX * 2));
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            // rotate the pieces across lanes (fewer bank conflicts); the
-                            // selects keep the data in registers
-                            const int p = (j + lane) & 3;
-                            const uint4 val = p == 0 ? u[0] : p == 1 ? u[1] : p == 2 ? u[2] : u[3];
-                            dst[p] = val;
-                        }
-                        fence_proxy_async_smem();
-                        __syncwarp();
-                        if (lane == 0) {
-                            tma_store_2d(&mOut, buf, col, c.a_row + q * 32);
-                            bulk_commit_group();
-                        }
-                        ++nstore;
-                    }
-                }
-            } else if (!c.shared) {
-                const int grow = c.a_row + row;
-                float wr;
-                __nv_bfloat16 *row_ptr;
-                int src = 0;
-                if (a.ep_P > 0) {
-                    // the row goes back to its token's rank, at the token's pair id;
-                    // padding rows carry source -1 and are not stored
-                    const int4 m = a.ep_meta[grow];
-                    src = (m.x >= 0 && m.x < a.ep_P) ? m.x : -1;
-                    wr = __int_as_float(m.z);
-                    row_ptr = src >= 0 ? a.ep_out[src] + (size_t)m.y * a.ld_r : nullptr;
-                } else {
-                    wr = a.w_perm[grow];
-                    row_ptr = a.out_r + (size_t)grow * a.ld_r;
-                }
-#pragma unroll 1
-                for (int ch = 0; ch < 8; ++ch) {
-                    uint32_t v[32];
-                    tmem_ld_32x32b_x32(tbase + ch * 32, v);
-                    tmem_ld_wait();
-                    const int col = c.nb * GEMM_BN + ch * 32;
-                    if (row_ptr && col < a.ncols_r) {
-                        float o[32];
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) o[i] = wr * __uint_as_float(v[i]);
-                        store_row_chunk_bf16(row_ptr, col, a.ncols_r, o);
-                    }
-                }
-                if (a.ep_P > 0) warp_count_rows(a.ep_ret, src, a.ep_P);
-            } else {
-                // shared expert: fp32 output rows, added last by combine_kernel
-                const int n = c.a_row + row;
-                float *row_ptr = a.osh + (size_t)n * a.ld_s;
-#pragma unroll 1
-                for (int ch = 0; ch < 8; ++ch) {
-                    uint32_t v[32];
-                    tmem_ld_32x32b_x32(tbase + ch * 32, v);
-                    tmem_ld_wait();
-                    const int col = c.nb * GEMM_BN + ch * 32;
-                    if (n < a.N && col < a.ncols_s) {
-#pragma unroll
-                        for (int qv = 0; qv < 8; ++qv)
-                            if (col + 4 * qv < a.ncols_s)
-                                reinterpret_cast<float4 *>(row_ptr + col)[qv] =
-                                    make_float4(__uint_as_float(v[4 * qv]), __uint_as_float(v[4 * qv + 1]),
-                                                __uint_as_float(v[4 * qv + 2]), __uint_as_float(v[4 * qv + 3]));
-                    }
-                }
-            }
+            epilogue_tile<KIND>(a, mOut, c, tbase, q, lane, stg, nstore);
             // Release the accumulator.
             tc_fence_before();
             __syncwarp();
@@ -588,6 +666,269 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, GEMM_TMEM_COLS);
+    }
+}
+
+}  // namespace moe
+
+namespace moe {
+
+// ---------------------------------------------------------------------------
+// The same grouped GEMMs on CTA pairs (cta_group::2).  A cluster of two CTAs
+// (the two SMs of a TPC) takes a pair tile: two consecutive m-tiles of one
+// expert (or of the shared expert) times one n-block.  CTA r loads its own 128
+// token rows (m-tile 2p + r) and half of the weight tile: gate_up the gate rows
+// (r = 0) or the matching up rows (r = 1), down the first or second 128 of the
+// 256 output features.  One thread of CTA 0 issues M = 256, N = 256, K = 16
+// MMAs over both CTAs' shared memory, and each CTA's TMEM receives the
+// accumulators of its own 128 rows: the same tile layout, so the same epilogue
+// as the one-CTA kernel.  Per k-block each SM loads 32 KiB instead of 48 KiB
+// for the same MMA work, so the ring holds six stages instead of four.
+//
+// Barriers: CTA 0's full[s] counts the bytes of both CTAs' loads (each CTA's
+// TMA completes on it; CTA 0 announces the total); every MMA batch's commit
+// arrives on empty[s] of both CTAs and the last one of a tile on tfull[acc] of
+// both; the eight epilogue warps of the pair release an accumulator on CTA 0's
+// tempty[acc].  Experts with an odd number of m-tiles leave their last m-tile
+// to the one-CTA kernel in GEMM_TAIL_TILES mode (so are the shared expert's
+// last m-tile when their count is odd); no MMA row is wasted on padding beyond
+// the 128-row segments.
+// ---------------------------------------------------------------------------
+constexpr int PAIR_STAGES = 6;
+constexpr int PAIR_A_BYTES = GEMM_BM * GEMM_BK * 2;  // 16 KiB: this CTA's 128 rows
+constexpr int PAIR_B_BYTES = 128 * GEMM_BK * 2;      // 16 KiB: this CTA's half of the 256 columns
+constexpr int PAIR_STAGE_BYTES = PAIR_A_BYTES + PAIR_B_BYTES;
+constexpr int PAIR_STG_OFF =
+    (PAIR_STAGES * PAIR_STAGE_BYTES + 256 + 2 * (GEMM_MAXE + 1) * 4 + 1023) / 1024 * 1024;
+constexpr int PAIR_SMEM_BYTES = 1024 + PAIR_STG_OFF + 4 * 2 * GEMM_OUT_BUF;
+static_assert(PAIR_SMEM_BYTES <= 232448, "shared memory");
+
+// Pair tile t for CTA `rank` of the pair: routed pairs first (expert-major,
+// n-block-major inside, so pairs that read the same weight tile run together),
+// then the shared expert's full pairs.  s_pair: prefix of m-tile pairs per expert.
+__device__ __forceinline__ TileCoord decode_pair(int t, int routed_tiles, const GemmArgs &a,
+                                                 const int *s_tile_off, const int *s_pair,
+                                                 int rank) {
+    TileCoord c;
+    if (t < routed_tiles) {
+        const int e = find_expert(s_pair, a.E, a.nb_r, t);
+        const int pe = s_pair[e + 1] - s_pair[e];
+        const int local = t - s_pair[e] * a.nb_r;
+        c.nb = local / pe;
+        const int p = local - c.nb * pe;
+        const int mt = s_tile_off[e] + 2 * p + rank;
+        c.valid = mt < s_tile_off[e + 1];
+        c.shared = false;
+        c.e = e;
+        c.a_row = mt * GEMM_BM;
+        c.kb = a.kb_r;
+    } else {
+        const int t2 = t - routed_tiles;
+        const int mp = t2 / a.nb_s;
+        c.nb = t2 - mp * a.nb_s;
+        c.valid = 2 * mp + (int)rank < a.mt_s;
+        c.shared = true;
+        c.e = -1;
+        c.a_row = (2 * mp + rank) * GEMM_BM;
+        c.kb = a.kb_s;
+    }
+    return c;
+}
+
+// Maps as grouped_gemm_kernel, with 128-row boxes for every B operand.
+template <int KIND>
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+    grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap mA_r,
+                             const __grid_constant__ CUtensorMap mB_r,
+                             const __grid_constant__ CUtensorMap mA_s,
+                             const __grid_constant__ CUtensorMap mB_s0,
+                             const __grid_constant__ CUtensorMap mB_s1,
+                             const __grid_constant__ CUtensorMap mOut, const GemmArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint8_t *ring = smem;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + PAIR_STAGES * PAIR_STAGE_BYTES);
+    uint64_t *empty = full + PAIR_STAGES;
+    uint64_t *tfull = empty + PAIR_STAGES;
+    uint64_t *tempty = tfull + 2;
+    uint64_t *drain = tempty + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    int *s_tile_off = reinterpret_cast<int *>(smem + PAIR_STAGES * PAIR_STAGE_BYTES + 256);
+    int *s_pair = s_tile_off + (GEMM_MAXE + 1);
+    // GEMM_PAIR_PAD: every m-tile runs here; an expert's odd last m-tile (and the
+    // shared expert's) forms a pair with an empty half, whose rows CTA 1 neither
+    // loads nor stores (its MMA rows are wasted).  Otherwise only full pairs run here.
+    const bool pad = a.mode == GEMM_PAIR_PAD;
+
+    const int warp = warp_id(), lane = lane_id();
+    const uint32_t rank = cluster_ctarank();
+    const int cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < PAIR_STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&tfull[i], 1);
+            mbar_init(&tempty[i], 8);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&mA_r);
+        tma_prefetch_desc(&mB_r);
+        tma_prefetch_desc(&mA_s);
+        tma_prefetch_desc(&mB_s0);
+        if (KIND == GEMM_GATE_UP) tma_prefetch_desc(&mB_s1);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(tmem_slot, GEMM_TMEM_COLS);
+        tmem_relinquish_pair();
+    }
+    for (int i = threadIdx.x; i <= a.E; i += blockDim.x) s_tile_off[i] = a.tile_off[i];
+    __syncthreads();
+    if (warp == 2) warp_expert_prefix(s_tile_off, a.E, s_pair, pad ? 2 : 0, lane);
+    tc_fence_before();
+    // Both CTAs' barriers are initialised and their TMEM allocated before either
+    // CTA's loads, MMAs or arrivals can reach the other.
+    cluster_sync_all();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const uint64_t limit = a.wait_limit_ns;
+    const int routed_tiles = s_pair[a.E] * a.nb_r;
+    const int total_tiles = routed_tiles + ((pad ? a.mt_s + 1 : a.mt_s) >> 1) * a.nb_s;
+
+    if (warp == 0) {
+        // ------------------------------ TMA producer (both CTAs) ------------------
+        if (lane == 0) {
+            uint32_t it = 0;
+            bool ok = true;
+            const uint32_t full0 = mapa_shared(smem_u32(full), 0); // CTA 0's full[0]
+            for (int t = cid; t < total_tiles && ok; t += ncl) {
+                const TileCoord c = decode_pair(t, routed_tiles, a, s_tile_off, s_pair, rank);
+                // bytes CTA 0 announces: both CTAs' operands less an empty half's rows
+                const bool full_pair = rank ? c.valid
+                                            : decode_pair(t, routed_tiles, a, s_tile_off, s_pair, 1).valid;
+                const uint32_t pair_bytes = 2 * PAIR_STAGE_BYTES - (full_pair ? 0 : PAIR_A_BYTES);
+                const CUtensorMap *mA = c.shared ? &mA_s : &mA_r;
+                const CUtensorMap *mB;
+                int brow;
+                if (KIND == GEMM_GATE_UP) {
+                    if (c.shared) {
+                        mB = rank ? &mB_s1 : &mB_s0;
+                        brow = c.nb * 128;
+                    } else {
+                        mB = &mB_r;
+                        brow = c.e * a.b_rows_per_e + (rank ? a.up_off : 0) + c.nb * 128;
+                    }
+                } else {
+                    mB = c.shared ? &mB_s0 : &mB_r;
+                    brow = (c.shared ? 0 : c.e * a.b_rows_per_e) + c.nb * GEMM_BN + rank * 128;
+                }
+                const int rot = c.nb % c.kb;
+                for (int i = 0; i < c.kb; ++i, ++it) {
+                    const int kb = i + rot < c.kb ? i + rot : i + rot - c.kb;
+                    const uint32_t s = it % PAIR_STAGES, ph = (it / PAIR_STAGES) & 1;
+                    if (!mbar_wait_cl(&empty[s], ph ^ 1, limit, abort_flag, 140)) { ok = false; break; }
+                    uint8_t *sa = ring + s * PAIR_STAGE_BYTES;
+                    if (rank == 0) mbar_arrive_expect_tx(&full[s], pair_bytes);
+                    const uint32_t fb = full0 + s * 8;
+                    const int kx = kb * GEMM_BK;
+                    if (c.valid) tma_load_2d_pair(mA, fb, sa, kx, c.a_row);
+                    tma_load_2d_pair(mB, fb, sa + PAIR_A_BYTES, kx, brow);
+                }
+            }
+            if (!ok && rank == 0) {
+                // Let copies already issued land before the pair's memory goes away.
+                const uint32_t first = it > PAIR_STAGES ? it - PAIR_STAGES : 0;
+                for (uint32_t j = first; j < it; ++j) {
+                    volatile int no_abort = 0;
+                    mbar_wait(&full[j % PAIR_STAGES], (j / PAIR_STAGES) & 1, 10000000ull, &no_abort, 141);
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------ MMA issuer (CTA 0) -------------------------
+        if (lane == 0 && rank == 0) {
+            constexpr uint32_t idesc = umma_idesc_bf16(2 * GEMM_BM, GEMM_BN);
+            uint32_t it = 0, tc = 0;
+            bool ok = true;
+            for (int t = cid; t < total_tiles && ok; t += ncl, ++tc) {
+                const TileCoord c = decode_pair(t, routed_tiles, a, s_tile_off, s_pair, 0);
+                const uint32_t acc = tc & 1, aph = (tc >> 1) & 1;
+                if (!mbar_wait_cl(&tempty[acc], aph ^ 1, limit, abort_flag, 150)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + acc * GEMM_BN;
+                for (int i = 0; i < c.kb; ++i, ++it) {
+                    const uint32_t s = it % PAIR_STAGES, ph = (it / PAIR_STAGES) & 1;
+                    if (!mbar_wait_cl(&full[s], ph, limit, abort_flag, 151)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t sa = smem_u32(ring + s * PAIR_STAGE_BYTES);
+                    const uint32_t sb = sa + PAIR_A_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < GEMM_BK / 16; ++kk)
+                        umma_bf16_ss_pair(d_tmem, umma_desc_sw128(sa + kk * 32),
+                                          umma_desc_sw128(sb + kk * 32), idesc,
+                                          (i > 0 || kk > 0) ? 1u : 0u);
+                    umma_commit_pair_mc(&empty[s], 0x3);
+                }
+                if (!ok) break;
+                umma_commit_pair_mc(&tfull[acc], 0x3);
+            }
+            // Drain: wait until every MMA issued by this thread has completed.
+            umma_commit_pair(drain);
+            volatile int no_abort = 0;
+            mbar_wait(drain, 0, 100000000ull, &no_abort, 152);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------ epilogue (both CTAs) -----------------------
+        const int q = warp & 3;
+        const int ep_tid = threadIdx.x - 64;
+        uint8_t *stg = smem + PAIR_STG_OFF + q * 2 * GEMM_OUT_BUF;
+        uint32_t nstore = 0;
+        uint32_t tc = 0;
+        const uint32_t tempty0 = mapa_shared(smem_u32(tempty), 0); // CTA 0's tempty[0]
+        for (int t = cid; t < total_tiles; t += ncl, ++tc) {
+            const TileCoord c = decode_pair(t, routed_tiles, a, s_tile_off, s_pair, rank);
+            const uint32_t acc = tc & 1, aph = (tc >> 1) & 1;
+            bool have = false;
+            if (lane == 0) have = mbar_wait_cl(&tfull[acc], aph, limit, abort_flag, 160);
+            have = __shfl_sync(0xffffffffu, have ? 1 : 0, 0) != 0;
+            __syncwarp();
+            if (have) {
+                tc_fence_after();
+                const uint32_t tbase = tmem_base + acc * GEMM_BN + ((uint32_t)(q * 32) << 16);
+                if (c.valid) epilogue_tile<KIND>(a, mOut, c, tbase, q, lane, stg, nstore);
+                // Release the accumulator to the pair's MMA issuer.
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_remote(tempty0 + acc * 8);
+            }
+            if (KIND == GEMM_DOWN) {
+                // Count the finished m-tile (combine_kernel checks the count).
+                __threadfence();
+                named_bar_sync(1, 128);
+                if (ep_tid == 0 && have && c.valid) atomicAdd(&a.meta[0], 1);
+            }
+        }
+    }
+
+    if (KIND == GEMM_DOWN && warp >= 2 && lane == 0) bulk_wait_group<0>(); // stores done
+    tc_fence_before();
+    // Neither CTA leaves while the pair's MMAs may still read its shared memory or
+    // the other CTA may still arrive on its barriers.
+    cluster_sync_all();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, GEMM_TMEM_COLS);
     }
 }
 

@@ -26,6 +26,10 @@ constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;
 constexpr int kDecodeMaxTokens = 256;
 uint64_t g_wait_limit_ns = kDefaultWaitLimitNs;
 int g_never_signal = 0;
+// Prefill expert GEMMs on CTA pairs: -1 (default) and 0 never, 1 full pairs with
+// the odd last m-tiles on the one-CTA kernel, 2 every m-tile in pairs, odd ones
+// with an empty half (a test and tuning hook).
+int g_pair_mode = -1;
 // Test hook: device buffer receiving the router's selection scores s' (null: off).
 float *g_dbg_sp = nullptr;
 size_t g_dbg_sp_n = 0;
@@ -70,6 +74,8 @@ struct DeviceInfo {
     int major, minor;
     bool gemm_attr_set;
     bool dec_attr_set;
+    bool pair_attr_set;
+    int pair_max_clusters; // co-resident CTA pairs of the pair kernels (0: unusable)
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -351,10 +357,16 @@ int launch_router_tc(const RouterParams &p, int sms, const RtcFuse &fz, bool pdl
     }
     const int tblocks = (p.N + RTC_BM - 1) / RTC_BM;
     // K-split cluster size: a power of two (so it divides the 128 tokens of a
-    // block) chosen to put about one CTA on every SM, at most 16 (8 where the
-    // device cannot co-schedule 16-CTA clusters of this kernel).
+    // block) chosen to put about one CTA on every SM, and large enough that no
+    // CTA accumulates more than RTC_MAX_KB k-blocks of the hidden dimension: the
+    // tensor core rounds toward zero at every accumulation step, so shorter
+    // chains (their partials summed in fp32 in rank order) keep the logits
+    // closer to the exact sum.  At most 16 (8 where the device cannot
+    // co-schedule 16-CTA clusters of this kernel).
+    const int KB = (p.D + RTC_BK - 1) / RTC_BK;
     int clk = 1;
-    while (clk < RTC_MAX_CLK && 2 * clk * tblocks <= sms) clk *= 2;
+    while (clk < RTC_MAX_CLK && (2 * clk * tblocks <= sms || (KB + clk - 1) / clk > RTC_MAX_KB))
+        clk *= 2;
     if (p.E <= 32) return launch_router_tc_t<1, WF32>(mX, mW, p, clk, fz, pdl, st);
     if (p.E <= 64) return launch_router_tc_t<2, WF32>(mX, mW, p, clk, fz, pdl, st);
     if (p.E <= 128) return launch_router_tc_t<4, WF32>(mX, mW, p, clk, fz, pdl, st);
@@ -376,6 +388,28 @@ int launch_gemm(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap 
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     if (cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<KIND>, a0, a1, a2, a3, a4, a5, args) !=
+        cudaSuccess)
+        return MOE_ERR_CUDA;
+    return launch_status();
+}
+
+template <int KIND>
+int launch_gemm_pair(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &a2,
+                     const CUtensorMap &a3, const CUtensorMap &a4, const CUtensorMap &a5,
+                     const GemmArgs &args, int clusters, cudaStream_t st) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * clusters, 1, 1);
+    cfg.blockDim = dim3(GEMM_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = PAIR_SMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, grouped_gemm_pair_kernel<KIND>, a0, a1, a2, a3, a4, a5, args) !=
         cudaSuccess)
         return MOE_ERR_CUDA;
     return launch_status();
@@ -429,6 +463,41 @@ int ensure_gemm_attrs(DeviceInfo *dev) {
                              GEMM_SMEM_BYTES) != cudaSuccess)
         return MOE_ERR_CUDA;
     dev->gemm_attr_set = true;
+    return MOE_OK;
+}
+
+// Shared-memory attributes of the pair kernels and the number of CTA pairs that
+// can be co-resident (0 if the device cannot run them; the one-CTA kernels then
+// take every tile).
+int ensure_pair_attrs(DeviceInfo *dev) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (dev->pair_attr_set) return MOE_OK;
+    dev->pair_max_clusters = 0;
+    if (cudaFuncSetAttribute(grouped_gemm_pair_kernel<GEMM_GATE_UP>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             PAIR_SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(grouped_gemm_pair_kernel<GEMM_DOWN>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             PAIR_SMEM_BYTES) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    cudaLaunchConfig_t q = {};
+    q.gridDim = dim3(2 * dev->sms, 1, 1);
+    q.blockDim = dim3(GEMM_THREADS, 1, 1);
+    q.dynamicSmemBytes = PAIR_SMEM_BYTES;
+    cudaLaunchAttribute qa[1];
+    qa[0].id = cudaLaunchAttributeClusterDimension;
+    qa[0].val.clusterDim.x = 2;
+    qa[0].val.clusterDim.y = 1;
+    qa[0].val.clusterDim.z = 1;
+    q.attrs = qa;
+    q.numAttrs = 1;
+    int c1 = 0, c2 = 0;
+    if (cudaOccupancyMaxActiveClusters(&c1, grouped_gemm_pair_kernel<GEMM_GATE_UP>, &q) ==
+            cudaSuccess &&
+        cudaOccupancyMaxActiveClusters(&c2, grouped_gemm_pair_kernel<GEMM_DOWN>, &q) == cudaSuccess)
+        dev->pair_max_clusters = std::min(c1, c2);
+    cudaGetLastError(); // a refused query only disables the pair kernels
+    dev->pair_attr_set = true;
     return MOE_OK;
 }
 
@@ -532,6 +601,12 @@ int moe_debug_set_wait_limit_ns(uint64_t ns) {
 
 int moe_debug_never_signal(int on) {
     g_never_signal = on ? 1 : 0;
+    return MOE_OK;
+}
+
+int moe_debug_set_pair_mode(int mode) {
+    if (mode < -1 || mode > 2) return MOE_ERR_ARG;
+    g_pair_mode = mode;
     return MOE_OK;
 }
 
@@ -797,7 +872,17 @@ int forward_impl(const void *x, const void *gate_up, const void *down, const voi
     }
 
     if ((rc = ensure_gemm_attrs(dev)) != MOE_OK) return rc;
-    CUtensorMap mx_perm, mgu, mx, msg, msu, mh_perm, mdn, mh_sh, msd;
+    // CTA pairs only on request: on the configurations measured (two to four
+    // m-tiles per expert on average) the pair kernels were not faster, because
+    // the odd last m-tiles either waste half an MMA tile or, in their own
+    // launch, stream their experts' weights from HBM a second time.
+    bool pair = g_pair_mode >= 1;
+    const bool pad = g_pair_mode == 2;
+    if (pair) {
+        if ((rc = ensure_pair_attrs(dev)) != MOE_OK) return rc;
+        pair = dev->pair_max_clusters > 0;
+    }
+    CUtensorMap mx_perm, mgu, mx, msg, msu, mh_perm, mdn, mh_sh, msd, mdn2, msd2;
     bool ok = make_map(&mx_perm, x_perm, D, L.rows_max, D, 128) &&
               make_map(&mgu, gate_up, D, (uint64_t)E * 2 * d_moe, D, 128) &&
               make_map(&mx, x, D, N, D, 128) && make_map(&msg, sh_gate, D, d_sh, D, 128) &&
@@ -805,7 +890,9 @@ int forward_impl(const void *x, const void *gate_up, const void *down, const voi
               make_map(&mh_perm, h_perm, d_moe, L.rows_max, d_moe, 128) &&
               make_map(&mdn, down, d_moe, (uint64_t)E * D, d_moe, GEMM_BN) &&
               make_map(&mh_sh, h_sh, d_sh, N, d_sh, 128) &&
-              make_map(&msd, sh_down, d_sh, D, d_sh, GEMM_BN);
+              make_map(&msd, sh_down, d_sh, D, d_sh, GEMM_BN) &&
+              (!pair || (make_map(&mdn2, down, d_moe, (uint64_t)E * D, d_moe, 128) &&
+                         make_map(&msd2, sh_down, d_sh, D, d_sh, 128)));
     if (!ok) return MOE_ERR_CUDA;
 
     const int mt_s = (N + GEMM_BM - 1) / GEMM_BM;
@@ -821,6 +908,10 @@ int forward_impl(const void *x, const void *gate_up, const void *down, const voi
     g.never_signal = g_never_signal;
     g.gate_max = gate_max;
     g.up_max = up_max;
+    // Launch sizes: the pair kernels take at most one pair tile per cluster; the
+    // tail launch has at most one m-tile per expert (and one shared m-tile).
+    const int pair_bound_mt = (mt_r_max + 1) / 2 + (mt_s + 1) / 2 + (pad ? E : 0);
+    const int tail_bound_mt = std::min(E, mt_r_max) + 1;
 
     // gate_up + SwiGLU
     g.nb_r = (d_moe + 127) / 128;
@@ -835,12 +926,25 @@ int forward_impl(const void *x, const void *gate_up, const void *down, const voi
     g.ld_s = d_sh;
     g.ncols_s = d_sh;
     int max_tiles = mt_r_max * g.nb_r + mt_s * g.nb_s;
-    rc = launch_gemm<GEMM_GATE_UP>(mx_perm, mgu, mx, msg, msu, mx, g,
-                                   std::min(dev->sms, max_tiles), false, st);
+    if (pair) {
+        const int nbm = std::max(g.nb_r, g.nb_s);
+        g.mode = pad ? GEMM_PAIR_PAD : GEMM_ALL_TILES;
+        rc = launch_gemm_pair<GEMM_GATE_UP>(mx_perm, mgu, mx, msg, msu, mx, g,
+                                            std::min(dev->pair_max_clusters,
+                                                     std::max(1, pair_bound_mt * nbm)), st);
+        if (rc != MOE_OK) return rc;
+        g.mode = GEMM_TAIL_TILES;
+        max_tiles = tail_bound_mt * nbm;
+    }
+    if (!pad) {
+        rc = launch_gemm<GEMM_GATE_UP>(mx_perm, mgu, mx, msg, msu, mx, g,
+                                       std::min(dev->sms, max_tiles), false, st);
+        if (rc != MOE_OK) return rc;
+    }
     prof.mark();
-    if (rc != MOE_OK) return rc;
 
     // down + weighted slot partials + shared expert + combine
+    g.mode = GEMM_ALL_TILES;
     g.nb_r = g.nb_s = (D + GEMM_BN - 1) / GEMM_BN;
     g.kb_r = (d_moe + GEMM_BK - 1) / GEMM_BK;
     g.kb_s = (d_sh + GEMM_BK - 1) / GEMM_BK;
@@ -860,10 +964,21 @@ int forward_impl(const void *x, const void *gate_up, const void *down, const voi
     CUtensorMap mslot;
     if (!make_map_out(&mslot, slot, D, L.rows_max, D)) return MOE_ERR_CUDA;
     max_tiles = mt_r_max * g.nb_r + mt_s * g.nb_s;
-    rc = launch_gemm<GEMM_DOWN>(mh_perm, mdn, mh_sh, msd, msd, mslot, g,
-                                std::min(dev->sms, max_tiles), false, st);
+    if (pair) {
+        g.mode = pad ? GEMM_PAIR_PAD : GEMM_ALL_TILES;
+        rc = launch_gemm_pair<GEMM_DOWN>(mh_perm, mdn2, mh_sh, msd2, msd2, mslot, g,
+                                         std::min(dev->pair_max_clusters,
+                                                  std::max(1, pair_bound_mt * g.nb_r)), st);
+        if (rc != MOE_OK) return rc;
+        g.mode = GEMM_TAIL_TILES;
+        max_tiles = tail_bound_mt * g.nb_r;
+    }
+    if (!pad) {
+        rc = launch_gemm<GEMM_DOWN>(mh_perm, mdn, mh_sh, msd, msd, mslot, g,
+                                    std::min(dev->sms, max_tiles), false, st);
+        if (rc != MOE_OK) return rc;
+    }
     prof.mark();
-    if (rc != MOE_OK) return rc;
     // y = slots in slot order + shared output, at many warps per SM
     combine_kernel<<<std::min((N + 7) / 8, dev->sms * 16), COMBINE_THREADS, 0, st>>>(g);
     return launched(prof);

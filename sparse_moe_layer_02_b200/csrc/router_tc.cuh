@@ -5,13 +5,15 @@
 // fp32.  fp32 W_g: every element is split into three bf16 parts,
 // w = w1 + w2 + w3 with w1 = bf16(w), w2 = bf16(w - w1), w3 = bf16(w - w1 - w2)
 // (each residual is exact in fp32, and the split reproduces w to 2^-27 relative,
-// finer than fp32 rounding), and x W_g^T is accumulated as three bf16 products
-// into the same fp32 accumulator.  Idle warps do the split into shared memory
-// while the TMA fetches the tokens.
+// finer than fp32 rounding), and x W_g^T is accumulated as three bf16 products:
+// the large part in one set of fp32 accumulators, the two small parts in
+// another.  Idle warps do the split into shared memory while the TMA fetches
+// the tokens.
 //
 // One cluster of CLK CTAs per 128 tokens: CTA r multiplies the tokens' rows by
 // W_g over the r-th slice of the hidden dimension (M = 128 tokens, N = E
-// experts, K = 16 per instruction; one 128 x E fp32 accumulator in TMEM).  The
+// experts, K = 16 per instruction; 128 x E fp32 accumulators in TMEM, k-blocks
+// rotating over several of them and summed in a fixed order at the end).  The
 // partial logits go to shared memory; after a cluster barrier, warps take whole
 // tokens, sum the CLK partial rows in rank order (distributed shared memory; a
 // fixed order, so the result is deterministic) and run the same warp-shuffle
@@ -34,6 +36,7 @@ constexpr int RTC_A_BYTES = RTC_BM * RTC_BK * 2;  // 16 KiB
 constexpr int RTC_PART_LD = 257;                  // floats per token row of the partials
 constexpr int RTC_MAXE_F32 = 192;                 // largest E of the fp32-W_g variant
 constexpr int RTC_MAX_CLK = 16;                   // largest K-split cluster (non-portable size)
+constexpr int RTC_MAX_KB = 24;                    // k-blocks per CTA above which K is split further
 
 template <bool WF32> struct RtcCfg {
     static constexpr int STAGES = WF32 ? 2 : 4;
@@ -148,7 +151,18 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
     const int KB = (p.D + RTC_BK - 1) / RTC_BK;
     const int kper = (KB + CLK - 1) / CLK;
     const int kb0 = rank * kper, kb1 = min(KB, kb0 + kper);
-    const uint32_t tmem_cols = E <= 32 ? 32 : E <= 64 ? 64 : E <= 128 ? 128 : 256;
+    // Accumulators: the 512 TMEM columns hold NA = 512 / ecols copies of the
+    // 128 x E logit tile.  Consecutive k-blocks rotate over NH of them (so each
+    // sums only every NH-th k-block), and for an fp32 W_g the two small bf16 parts
+    // of the split go to NL accumulators of their own, away from the large part.
+    // Every tensor-core accumulation step rounds at the magnitude of its
+    // accumulator; fewer steps per accumulator keep the logits closer to the
+    // exact sum.  The partials are added in a fixed order at the drain.
+    const uint32_t ecols = E <= 32 ? 32 : E <= 64 ? 64 : E <= 128 ? 128 : 256;
+    const uint32_t tmem_cols = 512;
+    const int NA = 512 / (int)ecols;
+    const int NH = WF32 ? NA / 2 : NA;
+    const int NL = WF32 ? NA / 2 : 0;
     // Every CTA reads the same W_g slices; rotating the k-block order by the token
     // block spreads concurrent reads over different L2 lines.
     const int nkb = kb1 > kb0 ? kb1 - kb0 : 0;
@@ -220,13 +234,21 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
                 tc_fence_after();
                 const uint32_t sa = smem_u32(ring + s * C::STAGE_BYTES);
                 const uint32_t sb = sa + RTC_A_BYTES;
+                const uint32_t dh = tmem_base + (uint32_t)(i % NH) * ecols;
+                const bool first_h = i < NH;
 #pragma unroll
                 for (int kk = 0; kk < RTC_BK / 16; ++kk) {
+                    umma_bf16_ss(dh, umma_desc_sw128(sa + kk * 32), umma_desc_sw128(sb + kk * 32),
+                                 idesc, (!first_h || kk > 0) ? 1u : 0u);
+                    if (WF32) {
+                        const uint32_t dl = tmem_base + (uint32_t)(NH + i % NL) * ecols;
+                        const bool first_l = i < NL;
 #pragma unroll
-                    for (int part_i = 0; part_i < (WF32 ? 3 : 1); ++part_i)
-                        umma_bf16_ss(tmem_base, umma_desc_sw128(sa + kk * 32),
-                                     umma_desc_sw128(sb + part_i * C::B_PART + kk * 32), idesc,
-                                     (i > 0 || kk > 0 || part_i > 0) ? 1u : 0u);
+                        for (int part_i = 1; part_i < 3; ++part_i)
+                            umma_bf16_ss(dl, umma_desc_sw128(sa + kk * 32),
+                                         umma_desc_sw128(sb + part_i * C::B_PART + kk * 32), idesc,
+                                         (!first_l || kk > 0 || part_i > 1) ? 1u : 0u);
+                    }
                 }
                 umma_commit(&empty[s]);
             }
@@ -295,16 +317,34 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
         have = __shfl_sync(0xffffffffu, have ? 1 : 0, 0) != 0;
         __syncwarp();
         if (have) tc_fence_after();
-        const bool empty_k = nkb == 0;
+        // Accumulators written by this CTA (a CTA with fewer k-blocks than NH leaves
+        // the others untouched); summed in a fixed order: large parts, then small.
+        const int nh = nkb < NH ? nkb : NH;
+        const int nl = nkb < NL ? nkb : NL;
+        const uint32_t lane_base = tmem_base + ((uint32_t)(q * 32) << 16);
         for (int c0 = 0; c0 < E; c0 += 32) {
-            uint32_t v[32];
+            float hi[32], lo[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) hi[i] = lo[i] = 0.f;
             if (have) {
-                tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + c0, v);
-                tmem_ld_wait();
+                for (int h = 0; h < nh; ++h) {
+                    uint32_t v[32];
+                    tmem_ld_32x32b_x32(lane_base + (uint32_t)h * ecols + c0, v);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) hi[i] = h ? hi[i] + __uint_as_float(v[i]) : __uint_as_float(v[i]);
+                }
+                for (int l = 0; l < nl; ++l) {
+                    uint32_t v[32];
+                    tmem_ld_32x32b_x32(lane_base + (uint32_t)(NH + l) * ecols + c0, v);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) lo[i] = l ? lo[i] + __uint_as_float(v[i]) : __uint_as_float(v[i]);
+                }
             }
 #pragma unroll
             for (int i = 0; i < 32; ++i)
-                if (c0 + i < E) part[row * RTC_PART_LD + c0 + i] = (have && !empty_k) ? __uint_as_float(v[i]) : 0.f;
+                if (c0 + i < E) part[row * RTC_PART_LD + c0 + i] = have ? hi[i] + lo[i] : 0.f;
         }
     }
     tc_fence_before();

@@ -124,6 +124,16 @@ def test_layer_call_rejects_bad_arguments_before_any_launch():
     assert call(N=0) == 0                  # no-op
 
 
+def test_debug_hooks_reject_bad_arguments():
+    lib = moe.load_library()
+    assert lib.moe_debug_set_pair_mode(3) == -1
+    assert lib.moe_debug_set_pair_mode(-2) == -1
+    assert lib.moe_debug_set_pair_mode(-1) == 0
+    assert lib.moe_debug_capture_scores(8, 16) == -1      # misaligned buffer
+    assert lib.moe_debug_capture_scores(16, 0) == -1      # empty buffer
+    assert lib.moe_debug_capture_scores(None, 0) == 0     # off
+
+
 def test_bias_update_rejects_bad_arguments():
     lib = moe.load_library()
     assert lib.moe_bias_update(None, 4, 2, 600, 1e-3, 16, None, None) == -2      # E > 512
