@@ -624,8 +624,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         __syncwarp();
     } else {
         // ------------------------------ epilogue ---------------------------------
-        const int q = warp & 3;          // TMEM lane quadrant of this warp
-        const int row = q * 32 + lane;   // row of the tile owned by this thread
+        const int q = warp & 3;          // TMEM lane quadrant of this warp (rows q*32 + lane)
         const int ep_tid = threadIdx.x - 64;
         uint8_t *stg = smem + GEMM_STG_OFF + q * 2 * GEMM_OUT_BUF; // this warp's two store buffers
         uint32_t nstore = 0;             // store boxes this warp has staged

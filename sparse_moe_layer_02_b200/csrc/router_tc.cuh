@@ -241,7 +241,7 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
                     umma_bf16_ss(dh, umma_desc_sw128(sa + kk * 32), umma_desc_sw128(sb + kk * 32),
                                  idesc, (!first_h || kk > 0) ? 1u : 0u);
                     if (WF32) {
-                        const uint32_t dl = tmem_base + (uint32_t)(NH + i % NL) * ecols;
+                        const uint32_t dl = tmem_base + (uint32_t)(NH + (NL > 0 ? i % NL : 0)) * ecols;
                         const bool first_l = i < NL;
 #pragma unroll
                         for (int part_i = 1; part_i < 3; ++part_i)
