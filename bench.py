@@ -75,9 +75,6 @@ def parse_args():
     ap.add_argument("--pair", default="off", choices=["off", "on", "pad"],
                     help="prefill expert GEMMs on CTA pairs: never (default), full pairs with "
                          "one-SM tails, padded pairs only")
-    ap.add_argument("--narrow-rows", type=int, default=64,
-                    help="largest last-m-tile row count run as a narrow (operand-swapped) tile "
-                         "by the one-SM prefill GEMMs; 0 = off")
     ap.add_argument("--graph", action="store_true",
                     help="capture the K timed steps as one CUDA graph and time one replay "
                          "(default: launch them one by one)")
@@ -711,7 +708,6 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=60), device_id=dev)
 
     moe.moe_debug_set_pair_mode({"off": 0, "on": 1, "pad": 2}[args.pair])
-    moe.moe_debug_set_narrow_rows(args.narrow_rows)
     cfg, over = workload(args.workload, args.set)
     head = measure(cfg, over, args, dev, dist, rank, world, local, moe, full=True)
     cpu, par = None, None
@@ -748,7 +744,6 @@ def main():
         "gpu_launches": head["gpu_launches"],
         "timing": head["timing"],
         "gemm_pairs": args.pair,
-        "narrow_rows": args.narrow_rows,
         "clocks": head["clocks"],
         "workloads": {
             name: {"value": res["value"], "unit": UNIT, "ms_per_step": res["ms_per_step"],

@@ -255,17 +255,6 @@ int moe_debug_never_signal(int on);
 int moe_debug_set_pair_mode(int mode);
 
 /*
- * Tuning and test hook for the one-SM prefill expert GEMMs: an expert's last
- * m-tile holding at most `rows` (0..64) token rows runs as a narrow tile, its
- * operands swapped (128 weight rows as the MMA's M, the token rows rounded up to
- * 16 as N), so the tensor cores skip the tile's padding rows.  0 turns narrow
- * tiles off; the default is 64.  The products and their order over K are the
- * same; the outputs agree with the normal tiles within rounding.  MOE_ERR_ARG for
- * values outside [0, 64].
- */
-int moe_debug_set_narrow_rows(int rows);
-
-/*
  * Test hook for the router's precision ("GLM-4.5 Group Router", How it works:
  * the gate runs in float32).  While buf is non-null, every router launch
  * (moe_router, moe_layer_forward) also writes each token's selection scores

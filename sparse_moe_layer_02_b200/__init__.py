@@ -21,7 +21,7 @@ __all__ = ["MoEError", "moe_router", "moe_forward", "moe_forward_workspace", "mo
            "moe_layer_forward_workspace",
            "moe_device_status", "moe_status_string", "moe_debug_set_wait_limit_ns",
            "moe_debug_never_signal", "moe_debug_capture_scores", "moe_debug_set_pair_mode",
-           "moe_debug_set_narrow_rows", "moe_profile_set_events",
+           "moe_profile_set_events",
            "moe_launch_count", "moe_forward_noalloc", "library_path", "load_library", "MOE_F32", "MOE_BF16",
            "EXPORTED_SYMBOLS", "moe_ep_symmetric_bytes", "moe_ep_workspace_bytes",
            "moe_ep_forward", "moe_ep_plan_host", "moe_ep_ipc_export", "moe_ep_ipc_open",
@@ -44,8 +44,7 @@ EXPORTED_SYMBOLS = ("moe_router", "moe_forward_workspace", "moe_layer_forward_wo
                     "moe_forward", "moe_device_status",
                     "moe_status_string", "moe_version", "moe_debug_set_wait_limit_ns",
                     "moe_debug_never_signal", "moe_profile_set_events", "moe_launch_count",
-                    "moe_debug_capture_scores", "moe_debug_set_pair_mode", "moe_debug_set_narrow_rows",
-                    "moe_forward_noalloc", "moe_forward_clamped", "moe_layer_forward",
+                    "moe_debug_capture_scores", "moe_debug_set_pair_mode", "moe_forward_noalloc", "moe_forward_clamped", "moe_layer_forward",
                     "moe_bias_update",
                     "moe_ep_symmetric_bytes",
                     "moe_ep_workspace_bytes", "moe_ep_forward", "moe_ep_plan_host",
@@ -92,8 +91,6 @@ def load_library():
         lib.moe_debug_set_wait_limit_ns.restype = I
         lib.moe_debug_never_signal.argtypes = [I]
         lib.moe_debug_never_signal.restype = I
-        lib.moe_debug_set_narrow_rows.argtypes = [I]
-        lib.moe_debug_set_narrow_rows.restype = I
         lib.moe_debug_set_pair_mode.argtypes = [I]
         lib.moe_debug_set_pair_mode.restype = I
         lib.moe_debug_capture_scores.argtypes = [P, ctypes.c_size_t]
@@ -331,12 +328,6 @@ def moe_debug_set_pair_mode(mode: int) -> None:
     """Prefill expert GEMMs on CTA pairs: 1 full pairs plus one-SM tails, 2 padded pairs
     only, 0 never, -1 automatic (default)."""
     _check(load_library().moe_debug_set_pair_mode(int(mode)), "moe_debug_set_pair_mode")
-
-
-def moe_debug_set_narrow_rows(rows: int) -> None:
-    """Largest last-m-tile row count run as a narrow (operand-swapped) tile by the
-    one-SM prefill GEMMs; 0 turns narrow tiles off (default 64)."""
-    _check(load_library().moe_debug_set_narrow_rows(int(rows)), "moe_debug_set_narrow_rows")
 
 
 def moe_debug_capture_scores(buf) -> None:

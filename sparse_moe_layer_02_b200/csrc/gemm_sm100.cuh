@@ -49,11 +49,7 @@ constexpr int GEMM_MAXE = 512;
 constexpr int GEMM_OUT_BOX = 32;                                   // rows and columns of a store box
 constexpr int GEMM_OUT_BUF = GEMM_OUT_BOX * GEMM_OUT_BOX * 2;     // 2 KiB
 constexpr int GEMM_STG_OFF =
-    (GEMM_STAGES * GEMM_STAGE_BYTES + 256 + 3 * (GEMM_MAXE + 1) * 4 + 1023) / 1024 * 1024;
-// Narrow tiles: token rows come in boxes of GEMM_NARROW_BOX rows; N is their count
-// rounded up to a multiple of GEMM_NARROW_BOX (a valid MMA N for M = 128).
-constexpr int GEMM_NARROW_BOX = 16;
-constexpr int GEMM_NARROW_MAX = 64;
+    (GEMM_STAGES * GEMM_STAGE_BYTES + 256 + 2 * (GEMM_MAXE + 1) * 4 + 1023) / 1024 * 1024;
 constexpr int GEMM_SMEM_BYTES = 1024 + GEMM_STG_OFF + 4 * 2 * GEMM_OUT_BUF;
 static_assert(GEMM_SMEM_BYTES <= 232448, "shared memory");
 
@@ -107,11 +103,6 @@ struct GemmArgs {
     // the last m-tile of every expert with an odd m-tile count (and the last shared
     // m-tile when their count is odd), the tiles the CTA-pair kernel leaves over.
     int mode;
-    // Narrow tiles (one-CTA kernel, single device): an expert's last m-tile holding
-    // at most narrow_max rows runs with the operands swapped, 128 weight rows as the
-    // MMA's M and its rows, rounded up to 16, as N.  0 = off.  counts: rows per expert.
-    int narrow_max;
-    const int32_t *counts;
     // Expert parallelism (all null / 0 for a single-device layer).  The routed
     // rows are other ranks' tokens received into this rank's buffer.
     const uint32_t *ep_wait_ctr;    // gate_up: rows arrived (this epoch) ...
@@ -129,7 +120,6 @@ struct TileCoord {
     int a_row; // row coordinate in the A map
     int nb;    // n-block
     int kb;    // k-blocks
-    int rows;  // narrow tile: the expert's real rows in it (1 .. a.narrow_max); 0 = a normal tile
 };
 
 // Exclusive prefix over the experts (one warp): out[e] = sum_{j < e} f(j) for
@@ -167,11 +157,9 @@ __device__ __forceinline__ int find_expert(const int *pre, int E, int nb, int t)
     return lo;
 }
 
-// s_aux: the tail prefix (warp_expert_prefix with kind 1) in GEMM_TAIL_TILES mode;
-// s_cnt: rows per expert (read only when narrow tiles are on).
+// s_aux: the tail prefix (warp_expert_prefix with odd = 1) in GEMM_TAIL_TILES mode.
 __device__ __forceinline__ TileCoord decode_tile(int t, int routed_tiles, const GemmArgs &a,
-                                                 const int *s_tile_off, const int *s_aux,
-                                                 const int *s_cnt) {
+                                                 const int *s_tile_off, const int *s_aux) {
     TileCoord c;
     if (t < routed_tiles) {
         if (a.mode == GEMM_TAIL_TILES) {
@@ -183,11 +171,6 @@ __device__ __forceinline__ TileCoord decode_tile(int t, int routed_tiles, const 
             c.e = e;
             c.a_row = (s_tile_off[e + 1] - 1) * GEMM_BM;
             c.kb = a.kb_r;
-            c.rows = 0;
-            if (a.narrow_max > 0) {
-                const int r = s_cnt[e] - (s_tile_off[e + 1] - s_tile_off[e] - 1) * GEMM_BM;
-                if (r <= a.narrow_max) c.rows = r;
-            }
             return c;
         }
         // Expert-major order: expert e owns tiles [tile_off[e] * nb_r, tile_off[e+1] * nb_r),
@@ -204,11 +187,6 @@ __device__ __forceinline__ TileCoord decode_tile(int t, int routed_tiles, const 
         c.e = lo;
         c.a_row = mt * GEMM_BM;
         c.kb = a.kb_r;
-        c.rows = 0;
-        if (a.narrow_max > 0 && mt == s_tile_off[lo + 1] - 1) {
-            const int r = s_cnt[lo] - (mte - 1) * GEMM_BM;
-            if (r <= a.narrow_max) c.rows = r;
-        }
     } else {
         const int t2 = t - routed_tiles;
         int mt;
@@ -224,7 +202,6 @@ __device__ __forceinline__ TileCoord decode_tile(int t, int routed_tiles, const 
         c.e = -1;
         c.a_row = mt * GEMM_BM;
         c.kb = a.kb_s;
-        c.rows = 0;
     }
     return c;
 }
@@ -479,48 +456,6 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs &a, const CUtensorM
     }
 }
 
-// Epilogue of a narrow tile (operands swapped): TMEM lane = feature, column =
-// token.  Thread `lane` of quadrant q owns feature f = q * 32 + lane of both
-// halves: gate_up reads the gate (columns 0..) and up (128..) projections of
-// feature nb * 128 + f and writes h = SwiGLU for each real row; down reads output
-// features nb * 256 + f and nb * 256 + 128 + f and writes them scaled by each row's
-// routing weight.  For a fixed row the 32 lanes of a warp store 32 consecutive
-// bf16 values.  Rows beyond c.rows (the padding of the last box) are not stored.
-template <int KIND>
-__device__ __forceinline__ void epilogue_narrow(const GemmArgs &a, const TileCoord &c,
-                                                uint32_t tbase, int q, int lane) {
-    const int f = q * 32 + lane;
-    for (int c0 = 0; c0 < c.rows; c0 += 32) {
-        uint32_t lo[32], hi[32];
-        tmem_ld_32x32b_x32(tbase + c0, lo);
-        tmem_ld_32x32b_x32(tbase + 128 + c0, hi);
-        tmem_ld_wait();
-        const int nr = min(32, c.rows - c0);
-        if (KIND == GEMM_GATE_UP) {
-            const int col = c.nb * 128 + f;
-            if (col < a.ncols_r) {
-                __nv_bfloat16 *out = a.out_r + (size_t)(c.a_row + c0) * a.ld_r + col;
-#pragma unroll
-                for (int t = 0; t < 32; ++t)
-                    if (t < nr)
-                        out[(size_t)t * a.ld_r] = __float2bfloat16_rn(
-                            swiglu_f(__uint_as_float(lo[t]), __uint_as_float(hi[t]), a.gate_max, a.up_max));
-            }
-        } else {
-            const int col0 = c.nb * GEMM_BN + f, col1 = col0 + 128;
-            __nv_bfloat16 *out = a.out_r + (size_t)(c.a_row + c0) * a.ld_r;
-#pragma unroll
-            for (int t = 0; t < 32; ++t) {
-                if (t < nr) {
-                    const float wr = a.w_perm[c.a_row + c0 + t];
-                    if (col0 < a.ncols_r) out[(size_t)t * a.ld_r + col0] = __float2bfloat16_rn(wr * __uint_as_float(lo[t]));
-                    if (col1 < a.ncols_r) out[(size_t)t * a.ld_r + col1] = __float2bfloat16_rn(wr * __uint_as_float(hi[t]));
-                }
-            }
-        }
-    }
-}
-
 // mOut (down with tma_out): the slot rows [rows, D] bf16, box 32 x 32, no swizzle.
 template <int KIND>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
@@ -529,8 +464,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                         const __grid_constant__ CUtensorMap mA_s,
                         const __grid_constant__ CUtensorMap mB_s0,
                         const __grid_constant__ CUtensorMap mB_s1,
-                        const __grid_constant__ CUtensorMap mOut,
-                        const __grid_constant__ CUtensorMap mA_n, const GemmArgs a) {
+                        const __grid_constant__ CUtensorMap mOut, const GemmArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -544,7 +478,6 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     int *s_tile_off = reinterpret_cast<int *>(smem + GEMM_STAGES * GEMM_STAGE_BYTES + 256);
     int *s_aux = s_tile_off + (GEMM_MAXE + 1);
-    int *s_cnt = s_aux + (GEMM_MAXE + 1);
 
     const int warp = warp_id(), lane = lane_id();
 
@@ -567,15 +500,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         tma_prefetch_desc(&mA_s);
         tma_prefetch_desc(&mB_s0);
         if (KIND == GEMM_GATE_UP) tma_prefetch_desc(&mB_s1);
-        if (a.narrow_max > 0) tma_prefetch_desc(&mA_n);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, GEMM_TMEM_COLS);
         tmem_relinquish();
     }
     for (int i = threadIdx.x; i <= a.E; i += blockDim.x) s_tile_off[i] = a.tile_off[i];
-    if (a.narrow_max > 0)
-        for (int i = threadIdx.x; i < a.E; i += blockDim.x) s_cnt[i] = a.counts[i];
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -615,7 +545,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             uint32_t it = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
-                const TileCoord c = decode_tile(t, routed_tiles, a, s_tile_off, s_aux, s_cnt);
+                const TileCoord c = decode_tile(t, routed_tiles, a, s_tile_off, s_aux);
                 const CUtensorMap *mA = c.shared ? &mA_s : &mA_r;
                 // Tiles of one n-block (same weight tile) start at the same k-block and
                 // share each weight line as it arrives; the n-blocks of one m-tile
@@ -628,18 +558,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     if (!mbar_wait(&empty[s], ph ^ 1, limit, abort_flag, 100)) { ok = false; break; }
                     uint8_t *sa = ring + s * GEMM_STAGE_BYTES;
                     uint8_t *sb = sa + GEMM_A_BYTES;
+                    mbar_arrive_expect_tx(&full[s], GEMM_STAGE_BYTES);
                     const int kx = kb * GEMM_BK;
-                    if (c.rows > 0) {
-                        // narrow tile: only the boxes of 16 token rows that hold real rows
-                        const int nbox = (c.rows + GEMM_NARROW_BOX - 1) / GEMM_NARROW_BOX;
-                        mbar_arrive_expect_tx(&full[s], GEMM_B_BYTES + nbox * GEMM_NARROW_BOX * GEMM_BK * 2);
-                        for (int j = 0; j < nbox; ++j)
-                            tma_load_2d(&mA_n, &full[s], sa + j * GEMM_NARROW_BOX * GEMM_BK * 2, kx,
-                                        c.a_row + j * GEMM_NARROW_BOX);
-                    } else {
-                        mbar_arrive_expect_tx(&full[s], GEMM_STAGE_BYTES);
-                        tma_load_2d(mA, &full[s], sa, kx, c.a_row);
-                    }
+                    tma_load_2d(mA, &full[s], sa, kx, c.a_row);
                     if (KIND == GEMM_GATE_UP) {
                         if (c.shared) {
                             tma_load_2d(&mB_s0, &full[s], sb, kx, c.nb * 128);
@@ -674,7 +595,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             uint32_t it = 0, tc = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++tc) {
-                const TileCoord c = decode_tile(t, routed_tiles, a, s_tile_off, s_aux, s_cnt);
+                const TileCoord c = decode_tile(t, routed_tiles, a, s_tile_off, s_aux);
                 const uint32_t acc = tc & 1, aph = (tc >> 1) & 1;
                 if (!mbar_wait(&tempty[acc], aph ^ 1, limit, abort_flag, 110)) { ok = false; break; }
                 tc_fence_after();
@@ -685,28 +606,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     tc_fence_after();
                     const uint32_t sa = smem_u32(ring + s * GEMM_STAGE_BYTES);
                     const uint32_t sb = sa + GEMM_A_BYTES;
-                    if (c.rows > 0) {
-                        // Narrow tile, operands swapped: D^T[feature, token] = W x^T.  The
-                        // weight tile's two 128-row halves (gate / up, or the first and
-                        // second 128 output features) are the M operands, the token rows
-                        // the N operand; accumulator columns [0, n) and [128, 128 + n).
-                        const int n = (c.rows + GEMM_NARROW_BOX - 1) / GEMM_NARROW_BOX * GEMM_NARROW_BOX;
-                        const uint32_t idn = umma_idesc_bf16(GEMM_BM, n);
 #pragma unroll
-                        for (int kk = 0; kk < GEMM_BK / 16; ++kk) {
-                            const uint64_t xdesc = umma_desc_sw128(sa + kk * 32);
-                            const uint32_t accf = (i > 0 || kk > 0) ? 1u : 0u;
-                            umma_bf16_ss(d_tmem, umma_desc_sw128(sb + kk * 32), xdesc, idn, accf);
-                            umma_bf16_ss(d_tmem + 128, umma_desc_sw128(sb + GEMM_B_BYTES / 2 + kk * 32),
-                                         xdesc, idn, accf);
-                        }
-                    } else {
-#pragma unroll
-                        for (int kk = 0; kk < GEMM_BK / 16; ++kk)
-                            umma_bf16_ss(d_tmem, umma_desc_sw128(sa + kk * 32),
-                                         umma_desc_sw128(sb + kk * 32), idesc,
-                                         (i > 0 || kk > 0) ? 1u : 0u);
-                    }
+                    for (int kk = 0; kk < GEMM_BK / 16; ++kk)
+                        umma_bf16_ss(d_tmem, umma_desc_sw128(sa + kk * 32),
+                                     umma_desc_sw128(sb + kk * 32), idesc,
+                                     (i > 0 || kk > 0) ? 1u : 0u);
                     umma_commit(&empty[s]);
                 }
                 if (!ok) break;
@@ -726,7 +630,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         uint32_t nstore = 0;             // store boxes this warp has staged
         uint32_t tc = 0;
         for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++tc) {
-            const TileCoord c = decode_tile(t, routed_tiles, a, s_tile_off, s_aux, s_cnt);
+            const TileCoord c = decode_tile(t, routed_tiles, a, s_tile_off, s_aux);
             const uint32_t acc = tc & 1, aph = (tc >> 1) & 1;
             // After an abort every wait fails at once; the loop still walks the same
             // tiles in every epilogue warp so the named barriers stay matched.
@@ -740,10 +644,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             tc_fence_after();
             const uint32_t tbase = tmem_base + acc * GEMM_BN + ((uint32_t)(q * 32) << 16);
 
-            if (c.rows > 0)
-                epilogue_narrow<KIND>(a, c, tbase, q, lane);
-            else
-                epilogue_tile<KIND>(a, mOut, c, tbase, q, lane, stg, nstore);
+            epilogue_tile<KIND>(a, mOut, c, tbase, q, lane, stg, nstore);
             // Release the accumulator.
             tc_fence_before();
             __syncwarp();
@@ -816,7 +717,6 @@ __device__ __forceinline__ TileCoord decode_pair(int t, int routed_tiles, const 
         const int p = local - c.nb * pe;
         const int mt = s_tile_off[e] + 2 * p + rank;
         c.valid = mt < s_tile_off[e + 1];
-        c.rows = 0;
         c.shared = false;
         c.e = e;
         c.a_row = mt * GEMM_BM;
@@ -826,7 +726,6 @@ __device__ __forceinline__ TileCoord decode_pair(int t, int routed_tiles, const 
         const int mp = t2 / a.nb_s;
         c.nb = t2 - mp * a.nb_s;
         c.valid = 2 * mp + (int)rank < a.mt_s;
-        c.rows = 0;
         c.shared = true;
         c.e = -1;
         c.a_row = (2 * mp + rank) * GEMM_BM;

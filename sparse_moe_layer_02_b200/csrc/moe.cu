@@ -26,9 +26,6 @@ constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;
 constexpr int kDecodeMaxTokens = 256;
 uint64_t g_wait_limit_ns = kDefaultWaitLimitNs;
 int g_never_signal = 0;
-// Rows up to which an expert's last m-tile runs as a narrow (operand-swapped) tile in
-// the one-SM prefill GEMMs; 0 = never (a test and tuning hook).
-int g_narrow_max = GEMM_NARROW_MAX;
 // Prefill expert GEMMs on CTA pairs: -1 (default) and 0 never, 1 full pairs with
 // the odd last m-tiles on the one-CTA kernel, 2 every m-tile in pairs, odd ones
 // with an empty half (a test and tuning hook).
@@ -376,13 +373,10 @@ int launch_router_tc(const RouterParams &p, int sms, const RtcFuse &fz, bool pdl
     return launch_router_tc_t<8, WF32>(mX, mW, p, clk, fz, pdl, st);
 }
 
-// a6: the token map with GEMM_NARROW_BOX-row boxes for narrow tiles (any map when
-// args.narrow_max is 0).
 template <int KIND>
 int launch_gemm(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &a2,
                 const CUtensorMap &a3, const CUtensorMap &a4, const CUtensorMap &a5,
-                const CUtensorMap &a6, const GemmArgs &args, int grid, bool cooperative,
-                cudaStream_t st) {
+                const GemmArgs &args, int grid, bool cooperative, cudaStream_t st) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid, 1, 1);
     cfg.blockDim = dim3(GEMM_THREADS, 1, 1);
@@ -393,7 +387,7 @@ int launch_gemm(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap 
     attr[0].val.cooperative = cooperative ? 1 : 0;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<KIND>, a0, a1, a2, a3, a4, a5, a6, args) !=
+    if (cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<KIND>, a0, a1, a2, a3, a4, a5, args) !=
         cudaSuccess)
         return MOE_ERR_CUDA;
     return launch_status();
@@ -607,12 +601,6 @@ int moe_debug_set_wait_limit_ns(uint64_t ns) {
 
 int moe_debug_never_signal(int on) {
     g_never_signal = on ? 1 : 0;
-    return MOE_OK;
-}
-
-int moe_debug_set_narrow_rows(int rows) {
-    if (rows < 0 || rows > GEMM_NARROW_MAX) return MOE_ERR_ARG;
-    g_narrow_max = rows;
     return MOE_OK;
 }
 
@@ -894,10 +882,8 @@ int forward_impl(const void *x, const void *gate_up, const void *down, const voi
         if ((rc = ensure_pair_attrs(dev)) != MOE_OK) return rc;
         pair = dev->pair_max_clusters > 0;
     }
-    CUtensorMap mx_perm, mgu, mx, msg, msu, mh_perm, mdn, mh_sh, msd, mdn2, msd2, mxn, mhn;
+    CUtensorMap mx_perm, mgu, mx, msg, msu, mh_perm, mdn, mh_sh, msd, mdn2, msd2;
     bool ok = make_map(&mx_perm, x_perm, D, L.rows_max, D, 128) &&
-              make_map(&mxn, x_perm, D, L.rows_max, D, GEMM_NARROW_BOX) &&
-              make_map(&mhn, h_perm, d_moe, L.rows_max, d_moe, GEMM_NARROW_BOX) &&
               make_map(&mgu, gate_up, D, (uint64_t)E * 2 * d_moe, D, 128) &&
               make_map(&mx, x, D, N, D, 128) && make_map(&msg, sh_gate, D, d_sh, D, 128) &&
               make_map(&msu, sh_up, D, d_sh, D, 128) &&
@@ -922,10 +908,6 @@ int forward_impl(const void *x, const void *gate_up, const void *down, const voi
     g.never_signal = g_never_signal;
     g.gate_max = gate_max;
     g.up_max = up_max;
-    // An expert's last m-tile with at most g_narrow_max rows runs as a narrow tile
-    // (one-SM kernels only; the pair kernels never narrow).
-    g.narrow_max = pair ? 0 : g_narrow_max;
-    g.counts = dp.counts;
     // Launch sizes: the pair kernels take at most one pair tile per cluster; the
     // tail launch has at most one m-tile per expert (and one shared m-tile).
     const int pair_bound_mt = (mt_r_max + 1) / 2 + (mt_s + 1) / 2 + (pad ? E : 0);
@@ -955,7 +937,7 @@ int forward_impl(const void *x, const void *gate_up, const void *down, const voi
         max_tiles = tail_bound_mt * nbm;
     }
     if (!pad) {
-        rc = launch_gemm<GEMM_GATE_UP>(mx_perm, mgu, mx, msg, msu, mx, mxn, g,
+        rc = launch_gemm<GEMM_GATE_UP>(mx_perm, mgu, mx, msg, msu, mx, g,
                                        std::min(dev->sms, max_tiles), false, st);
         if (rc != MOE_OK) return rc;
     }
@@ -992,7 +974,7 @@ int forward_impl(const void *x, const void *gate_up, const void *down, const voi
         max_tiles = tail_bound_mt * g.nb_r;
     }
     if (!pad) {
-        rc = launch_gemm<GEMM_DOWN>(mh_perm, mdn, mh_sh, msd, msd, mslot, mhn, g,
+        rc = launch_gemm<GEMM_DOWN>(mh_perm, mdn, mh_sh, msd, msd, mslot, g,
                                     std::min(dev->sms, max_tiles), false, st);
         if (rc != MOE_OK) return rc;
     }
@@ -1274,7 +1256,7 @@ int ep_forward_impl(int phases, int P, int rank, uint32_t epoch, void *const *pe
         g.ep_wait_ctr = reinterpret_cast<const uint32_t *>(own + S.ctr) + par;
         g.ep_wait_target = ep.rmeta + 3;
         int max_tiles = mt_r_max * g.nb_r + mt_s * g.nb_s;
-        rc = launch_gemm<GEMM_GATE_UP>(mx_perm, mgu, mx, msg, msu, mx, mx, g,
+        rc = launch_gemm<GEMM_GATE_UP>(mx_perm, mgu, mx, msg, msu, mx, g,
                                        std::min(dev->sms, max_tiles), false, st);
         prof.mark();
         if (rc != MOE_OK) return rc;
@@ -1297,7 +1279,7 @@ int ep_forward_impl(int phases, int P, int rank, uint32_t epoch, void *const *pe
             g.ep_ret[q] = reinterpret_cast<uint32_t *>(ep.sym[q] + S.ctr) + 2 + par;
         }
         max_tiles = mt_r_max * g.nb_r + mt_s * g.nb_s;
-        rc = launch_gemm<GEMM_DOWN>(mh_perm, mdn, mh_sh, msd, msd, msd, msd, g,
+        rc = launch_gemm<GEMM_DOWN>(mh_perm, mdn, mh_sh, msd, msd, msd, g,
                                     std::min(dev->sms, max_tiles), true, st);
         prof.mark();
         if (rc != MOE_OK) return rc;

@@ -129,9 +129,6 @@ def test_debug_hooks_reject_bad_arguments():
     assert lib.moe_debug_set_pair_mode(3) == -1
     assert lib.moe_debug_set_pair_mode(-2) == -1
     assert lib.moe_debug_set_pair_mode(-1) == 0
-    assert lib.moe_debug_set_narrow_rows(65) == -1
-    assert lib.moe_debug_set_narrow_rows(-1) == -1
-    assert lib.moe_debug_set_narrow_rows(64) == 0
     assert lib.moe_debug_capture_scores(8, 16) == -1      # misaligned buffer
     assert lib.moe_debug_capture_scores(16, 0) == -1      # empty buffer
     assert lib.moe_debug_capture_scores(None, 0) == 0     # off

@@ -9,9 +9,8 @@ ever waits for another one that is still running.
 The expert rows go through the same prefill kernels, with the same operand rows,
 weights and k-block order as on one device, so each rank's y must equal
 moe_forward's on that rank's tokens bit for bit (token counts above 256, where
-moe_forward takes those kernels, with its narrow tail tiles off: the expert-parallel
-path runs every tile with tokens as the MMA's M operand); smaller batches are
-compared within the bf16 bound, and one rank against the oracle.
+moe_forward takes those kernels); smaller batches are compared within the bf16
+bound, and one rank against the oracle.
 """
 
 import numpy as np
@@ -32,10 +31,8 @@ DEV = "cuda:0"
 @pytest.fixture(autouse=True)
 def _reset_hooks():
     moe.moe_debug_set_wait_limit_ns(0)
-    moe.moe_debug_set_narrow_rows(0)
     yield
     moe.moe_debug_set_wait_limit_ns(0)
-    moe.moe_debug_set_narrow_rows(64)
 
 
 class _Ranks:

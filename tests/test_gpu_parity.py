@@ -296,13 +296,11 @@ def test_pair_gemms_match_oracle_and_single_cta(case):
     w = torch.from_numpy(orc["w"]).float().to(DEV)
     ys = {}
     try:
-        moe.moe_debug_set_narrow_rows(0)  # the one-SM baseline without narrow tiles
         for mode in (1, 2, 0):
             moe.moe_debug_set_pair_mode(mode)
             ys[mode] = _gpu_forward(d, idx, w)
     finally:
         moe.moe_debug_set_pair_mode(-1)
-        moe.moe_debug_set_narrow_rows(64)
     for mode in (1, 2):
         err = rel_err(ys[mode].float().cpu().numpy(), y_ref)
         print(case, mode, err)
@@ -319,60 +317,12 @@ def test_pair_gemms_full_size_equal_single_cta(name):
                             cfg.norm_topk_prob, cfg.alpha)
     ys = {}
     try:
-        moe.moe_debug_set_narrow_rows(0)
         for mode in (1, 2, 0):
             moe.moe_debug_set_pair_mode(mode)
             ys[mode] = _gpu_forward(inp, idx, w)
     finally:
         moe.moe_debug_set_pair_mode(-1)
-        moe.moe_debug_set_narrow_rows(64)
     assert torch.equal(ys[1], ys[0]) and torch.equal(ys[2], ys[0])
-
-
-# ----------------------------------------------------------------- narrow tail tiles
-NARROW_CASES = {
-    # every expert's last m-tile narrow or not, rows 1..64 and above: 40 experts of
-    # loads spread over 1..400 rows (hand-made routing)
-    "narrow_spread": dict(N=700, D=520, E=40, k=8, d_moe=200, d_sh=136),
-    # D and d_moe multiples of the tiles, a few tokens per expert (all tails narrow)
-    "narrow_small_loads": dict(N=300, D=512, E=64, k=4, d_moe=256, d_sh=256),
-}
-
-
-@pytest.mark.parametrize("case", list(NARROW_CASES))
-def test_narrow_tail_tiles(case):
-    """An expert's last m-tile with at most 64 rows runs with the operands swapped
-    (weights as the MMA's M, its rows as N).  Against the oracle, and against the
-    same layer with narrow tiles off, within the bf16 bound; the test also prints
-    whether the two agree bit for bit."""
-    cfg = CONFIGS["glm5_prefill"].with_(**NARROW_CASES[case])
-    inp = make_inputs(cfg, seed=21, device="cpu")
-    rng = np.random.default_rng(5)
-    # loads: expert e gets about 10 * e + 1 (token, slot) pairs -> tails of every size
-    p = np.arange(1, cfg.E + 1, dtype=np.float64)
-    p = p / p.sum()
-    idx = np.stack([rng.choice(cfg.E, size=cfg.k, replace=False, p=p) for _ in range(cfg.N)])
-    idx = idx.astype(np.int32)
-    w = rng.uniform(0.1, 1.0, size=idx.shape)
-    loads = np.bincount(idx.ravel(), minlength=cfg.E)
-    tails = loads - 128 * np.maximum((loads + 127) // 128 - 1, 0)
-    assert (tails[loads > 0] <= 64).any() and (tails[loads > 0] > 64).any() or case != "narrow_spread"
-    y_ref = oracle.forward(*_weights(inp), idx, w)
-    d = inp.to(DEV)
-    di, dw = torch.from_numpy(idx).to(DEV), torch.from_numpy(w).float().to(DEV)
-    try:
-        moe.moe_debug_set_narrow_rows(0)
-        y_off = _gpu_forward(d, di, dw)
-    finally:
-        moe.moe_debug_set_narrow_rows(64)
-    y_on = _gpu_forward(d, di, dw)
-    for y in (y_on, y_off):
-        err = rel_err(y.float().cpu().numpy(), y_ref)
-        assert err["finite"] and err["max_rel"] <= Y_TOL[cfg.dtype], err
-        assert err["max_row_l2_rel"] <= Y_TOL[cfg.dtype], err
-    diff = rel_err(y_on.float().cpu().numpy(), y_off.float().cpu().numpy())
-    print(case, "narrow on vs off:", diff, "bit-identical:", bool(torch.equal(y_on, y_off)))
-    assert diff["max_rel"] <= Y_TOL[cfg.dtype]
 
 
 # ----------------------------------------------------------------------------- full size
