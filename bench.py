@@ -260,9 +260,9 @@ def roofline_of(cfg, name: str, hit: int, ms: float, peaks: dict, peak_src: str)
     roof["kernel"] = name
     roof["ms_per_launch"] = ms
     roof["algorithmic"] = {"flops": flops, "bytes": byts}
-    roof["north_star"] = {
+    roof["vs_nominal"] = {
         "peak": nominal, "unit": roof["unit"], "frac": roof["achieved"] / nominal,
-        "target": TARGET[roof["bound"]],
+        "target": TARGET[roof["bound"]], "target_is_judged_on_this_fraction": True,
         "what": ("the layer's stated target: prefill grouped GEMMs >= 60 % of the nominal "
                  "dense bf16 peak (2.25 PFLOP/s)" if roof["bound"] == "tensor" else
                  "the layer's stated target: decode >= 70 % of ~8 TB/s over the hit "

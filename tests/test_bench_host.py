@@ -48,13 +48,13 @@ def test_roofline_arithmetic():
     assert r["bound"] == "tensor"
     assert r["achieved"] == pytest.approx(flops / 5e-3 / 1e12)
     assert r["frac"] == pytest.approx(r["achieved"] / 1200.0)
-    assert r["north_star"]["frac"] == pytest.approx(r["achieved"] / 2250.0)
-    assert r["north_star"]["target"] == 0.60
+    assert r["vs_nominal"]["frac"] == pytest.approx(r["achieved"] / 2250.0)
+    assert r["vs_nominal"]["target"] == 0.60
     dec = CONFIGS["air_decode"]
     r = bench.roofline_of(dec, "gate_up_swiglu", 100, 0.4, peaks, "fallback")
     assert r["bound"] == "hbm" and r["unit"] == "GB/s"
-    assert r["north_star"]["frac"] == pytest.approx(r["achieved"] / 8000.0)
-    assert r["north_star"]["target"] == 0.70
+    assert r["vs_nominal"]["frac"] == pytest.approx(r["achieved"] / 8000.0)
+    assert r["vs_nominal"]["target"] == 0.70
     assert r["peak_source"] == "fallback copy"
 
 
