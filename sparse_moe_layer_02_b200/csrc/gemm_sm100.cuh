@@ -36,6 +36,8 @@ namespace moe {
 constexpr int GEMM_BM = 128;
 constexpr int GEMM_BN = 256;
 constexpr int GEMM_BK = 64;
+// Four 48 KiB stages: the most that fit beside the store staging.  The main loop
+// is sensitive to the depth (three stages made gate_up 7 % slower).
 constexpr int GEMM_STAGES = 4;
 constexpr int GEMM_THREADS = 192;
 constexpr int GEMM_A_BYTES = GEMM_BM * GEMM_BK * 2;  // 16 KiB
@@ -688,10 +690,12 @@ namespace moe {
 // TMA completes on it; CTA 0 announces the total); every MMA batch's commit
 // arrives on empty[s] of both CTAs and the last one of a tile on tfull[acc] of
 // both; the eight epilogue warps of the pair release an accumulator on CTA 0's
-// tempty[acc].  Experts with an odd number of m-tiles leave their last m-tile
-// to the one-CTA kernel in GEMM_TAIL_TILES mode (so are the shared expert's
-// last m-tile when their count is odd); no MMA row is wasted on padding beyond
-// the 128-row segments.
+// tempty[acc].  An expert with an odd number of m-tiles either leaves its last
+// m-tile to the one-CTA kernel in GEMM_TAIL_TILES mode (as does the shared
+// expert's last m-tile when their count is odd) or, in GEMM_PAIR_PAD mode, runs
+// it here as a pair whose second half has no rows (its MMA rows are wasted).
+// Measured on the prefill configurations, neither beat the one-CTA kernel alone,
+// so these kernels run only on request (moe_debug_set_pair_mode).
 // ---------------------------------------------------------------------------
 constexpr int PAIR_STAGES = 6;
 constexpr int PAIR_A_BYTES = GEMM_BM * GEMM_BK * 2;  // 16 KiB: this CTA's 128 rows
