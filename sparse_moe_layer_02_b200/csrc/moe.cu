@@ -877,11 +877,12 @@ int forward_impl(const void *x, const void *gate_up, const void *down, const voi
     // the odd last m-tiles either waste half an MMA tile or, in their own
     // launch, stream their experts' weights from HBM a second time.
     bool pair = g_pair_mode >= 1;
-    const bool pad = g_pair_mode == 2;
     if (pair) {
         if ((rc = ensure_pair_attrs(dev)) != MOE_OK) return rc;
         pair = dev->pair_max_clusters > 0;
     }
+    // padded pairs take every m-tile (no one-CTA launch); only if pairs can run
+    const bool pad = pair && g_pair_mode == 2;
     CUtensorMap mx_perm, mgu, mx, msg, msu, mh_perm, mdn, mh_sh, msd, mdn2, msd2;
     bool ok = make_map(&mx_perm, x_perm, D, L.rows_max, D, 128) &&
               make_map(&mgu, gate_up, D, (uint64_t)E * 2 * d_moe, D, 128) &&
