@@ -88,6 +88,39 @@ def test_router_bias_reorders_selection_but_not_weights():
     assert rep["unexplained"] == 0 and rep["max_w_err_over_alpha"] <= W_TOL
 
 
+@pytest.mark.parametrize("x_dtype", [torch.bfloat16, torch.float32])
+def test_router_exact_ties_go_to_the_lower_index(x_dtype):
+    """Exact ties, decided the same way on both sides: every expert has a twin with
+    an identical router row and bias (so bitwise-equal logits on the GPU and equal
+    scores in the oracle), and groups 1 and 3 copy groups 0 and 2 (equal group
+    scores; one group is kept, so a group tie sits at the boundary).  Lower ids and
+    lower groups win, so the ids must equal the oracle's exactly, order included,
+    with no near-tie allowance."""
+    cfg = CONFIGS["skew_grouped"].with_(N=256, D=256, E=32, n_group=4, topk_group=1, k=3,
+                                        skew=False)
+    x, wg, b, _ = router_inputs(cfg, seed=17, device=DEV)
+    x = x.to(x_dtype)
+    wg = wg.clone()
+    b = b.clone()
+    for g in (1, 3):                     # group g copies group g - 1 (8 experts each)
+        wg[8 * g:8 * g + 8] = wg[8 * (g - 1):8 * g]
+        b[8 * g:8 * g + 8] = b[8 * (g - 1):8 * g]
+    wg[1::2] = wg[0::2]                  # every odd expert copies its even neighbour
+    b[1::2] = b[0::2]
+    W_g = wg.to(torch.bfloat16) if x_dtype == torch.bfloat16 else wg
+    idx, w = moe.moe_router(x, W_g, b, cfg.n_group, cfg.topk_group, cfg.k, True, cfg.alpha)
+    assert moe.moe_device_status() == 0
+    orc = oracle.router(x.cpu(), W_g.cpu(), b.cpu(), cfg.n_group, cfg.topk_group, cfg.k, True,
+                        cfg.alpha)
+    np.testing.assert_array_equal(idx.cpu().numpy(), orc["idx"])
+    # ties at both boundaries did occur: a chosen expert's twin left out, and only
+    # the even group of each tied pair kept
+    gi = idx.cpu().numpy()
+    assert any((e ^ 1) not in row for row in gi for e in row)
+    assert set((gi // 8).ravel().tolist()) <= {0, 2}
+    assert np.max(np.abs(w.cpu().double().numpy() - orc["w"])) / cfg.alpha <= W_TOL
+
+
 @pytest.mark.parametrize("E,G,tg,k", [(64, 8, 3, 6), (512, 1, 1, 8), (288, 1, 1, 8),
                                       (256, 64, 8, 16), (160, 1, 1, 1)])
 def test_router_shapes(E, G, tg, k):
