@@ -56,6 +56,18 @@ F32_KERNELS = ["dispatch_count", "dispatch_scan", "dispatch_scatter", "gate_up_r
                "gate_up_shared", "down_routed", "down_shared", "combine"]
 
 
+# What each --pair setting runs for the prefill expert GEMMs (moe_debug_set_pair_mode).
+PAIR_MODES = {
+    "default": "library default: down on CTA pairs for experts with an even m-tile count, "
+               "the rest and all of gate_up on one SM",
+    "off": "every tile on one SM",
+    "on": "CTA pairs, odd last m-tiles on one SM",
+    "pad": "CTA pairs, odd last m-tiles padded",
+    "parity": "gate_up and down on CTA pairs for experts with an even m-tile count",
+    "down": "down on CTA pairs for experts with an even m-tile count, gate_up on one SM",
+}
+
+
 def parse_args():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -72,9 +84,11 @@ def parse_args():
                     help="target duration of the oracle's CPU-baseline sample")
     ap.add_argument("--set", action="append", default=[], metavar="FIELD=VALUE",
                     help="override a size of the workload (e.g. E=32) for small profiling cases")
-    ap.add_argument("--pair", default="off", choices=["off", "on", "pad"],
-                    help="prefill expert GEMMs on CTA pairs: never (default), full pairs with "
-                         "one-SM tails, padded pairs only")
+    ap.add_argument("--pair", default="default",
+                    choices=["default", "off", "on", "pad", "parity", "down"],
+                    help="prefill expert GEMMs on CTA pairs: the library's default, never, "
+                         "full pairs with one-SM tails, padded pairs only, even-count experts "
+                         "on pairs and the rest on one SM, or that split for down only")
     ap.add_argument("--graph", action="store_true",
                     help="capture the K timed steps as one CUDA graph and time one replay "
                          "(default: launch them one by one)")
@@ -707,7 +721,8 @@ def main():
 
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=60), device_id=dev)
 
-    moe.moe_debug_set_pair_mode({"off": 0, "on": 1, "pad": 2}[args.pair])
+    moe.moe_debug_set_pair_mode(
+        {"default": -1, "off": 0, "on": 1, "pad": 2, "parity": 3, "down": 4}[args.pair])
     cfg, over = workload(args.workload, args.set)
     head = measure(cfg, over, args, dev, dist, rank, world, local, moe, full=True)
     cpu, par = None, None
@@ -743,7 +758,7 @@ def main():
         "e2e": head["e2e"],
         "gpu_launches": head["gpu_launches"],
         "timing": head["timing"],
-        "gemm_pairs": args.pair,
+        "gemm_pairs": PAIR_MODES[args.pair],
         "clocks": head["clocks"],
         "workloads": {
             name: {"value": res["value"], "unit": UNIT, "ms_per_step": res["ms_per_step"],

@@ -247,10 +247,11 @@ int moe_debug_never_signal(int on);
  * tokens).  Mode 1 runs them on CTA pairs (two SMs share one M = 256
  * tensor-core tile) with the odd last m-tile of each expert on the one-SM
  * kernels; mode 2 runs every m-tile on CTA pairs, an odd last m-tile pairing
- * with an empty half; modes 0 and -1 (the default) run every tile on the
- * one-SM kernels, which were the faster ones on every configuration measured.
- * Results are identical bit for bit in every mode.  MOE_ERR_ARG for other
- * values.
+ * with an empty half; mode 3 runs the experts with an even number of m-tiles
+ * on CTA pairs and the others on the one-SM kernels; mode 4 does that for the
+ * down GEMM only; mode 0 runs every tile on the one-SM kernels; -1 restores
+ * the library's default (mode 4).  Results are identical bit for bit in every
+ * mode.  MOE_ERR_ARG for other values.
  */
 int moe_debug_set_pair_mode(int mode);
 

@@ -326,7 +326,8 @@ def moe_debug_never_signal(on: bool):
 
 def moe_debug_set_pair_mode(mode: int) -> None:
     """Prefill expert GEMMs on CTA pairs: 1 full pairs plus one-SM tails, 2 padded pairs
-    only, 0 never, -1 automatic (default)."""
+    only, 3 even-count experts on pairs and the rest on one SM, 4 that split for the down
+    GEMM only, 0 never; -1 restores the library's default."""
     _check(load_library().moe_debug_set_pair_mode(int(mode)), "moe_debug_set_pair_mode")
 
 

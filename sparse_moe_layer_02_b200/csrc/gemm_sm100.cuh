@@ -56,7 +56,13 @@ constexpr int GEMM_SMEM_BYTES = 1024 + GEMM_STG_OFF + 4 * 2 * GEMM_OUT_BUF;
 static_assert(GEMM_SMEM_BYTES <= 232448, "shared memory");
 
 enum GemmKind { GEMM_GATE_UP = 0, GEMM_DOWN = 1 };
-enum GemmTiles { GEMM_ALL_TILES = 0, GEMM_TAIL_TILES = 1, GEMM_PAIR_PAD = 2 };
+enum GemmTiles {
+    GEMM_ALL_TILES = 0,   // one-CTA kernel: every tile; pair kernel: every full pair
+    GEMM_TAIL_TILES = 1,  // one-CTA kernel: the odd last m-tile of each expert
+    GEMM_PAIR_PAD = 2,    // pair kernel: every m-tile, an odd last one with an empty half
+    GEMM_ODD_EXPERTS = 3, // one-CTA kernel: every tile of the experts with an odd m-tile count
+    GEMM_EVEN_EXPERTS = 4 // pair kernel: every tile of the experts with an even m-tile count
+};
 
 constexpr int EP_MAX_RANKS = 8; // ranks of an expert-parallel group
 
@@ -127,7 +133,8 @@ struct TileCoord {
 // Exclusive prefix over the experts (one warp): out[e] = sum_{j < e} f(j) for
 // e in [0, E], with f(j) from expert j's m-tile count m (tile prefix tile_off):
 // kind 0 the full pairs m / 2, kind 1 the odd tail m % 2, kind 2 the pairs
-// including a half-empty last one, (m + 1) / 2.
+// including a half-empty last one, (m + 1) / 2, kind 3 all m-tiles of an odd
+// count (0 for even), kind 4 the pairs of an even count (0 for odd).
 __device__ __forceinline__ void warp_expert_prefix(const int *tile_off, int E, int *out, int kind,
                                                    int lane) {
     int carry = 0;
@@ -136,7 +143,11 @@ __device__ __forceinline__ void warp_expert_prefix(const int *tile_off, int E, i
         int v = 0;
         if (e < E) {
             const int m = tile_off[e + 1] - tile_off[e];
-            v = kind == 1 ? (m & 1) : kind == 2 ? ((m + 1) >> 1) : (m >> 1);
+            v = kind == 1 ? (m & 1)
+                : kind == 2 ? ((m + 1) >> 1)
+                : kind == 3 ? ((m & 1) ? m : 0)
+                : kind == 4 ? ((m & 1) ? 0 : (m >> 1))
+                : (m >> 1);
         }
         int incl = v;
 #pragma unroll
@@ -178,10 +189,12 @@ __device__ __forceinline__ TileCoord decode_tile(int t, int routed_tiles, const 
         // Expert-major order: expert e owns tiles [tile_off[e] * nb_r, tile_off[e+1] * nb_r),
         // n-block-major inside, so the m-tiles that read the same weight tile are
         // neighbours in the round-robin and run at the same time (one HBM read,
-        // the others hit L2).
-        const int lo = find_expert(s_tile_off, a.E, a.nb_r, t);
+        // the others hit L2).  GEMM_ODD_EXPERTS numbers only the odd-count experts'
+        // tiles, through their prefix s_aux, in the same order.
+        const int *pre = a.mode == GEMM_ODD_EXPERTS ? s_aux : s_tile_off;
+        const int lo = find_expert(pre, a.E, a.nb_r, t);
         const int mte = s_tile_off[lo + 1] - s_tile_off[lo];
-        const int local = t - s_tile_off[lo] * a.nb_r;
+        const int local = t - pre[lo] * a.nb_r;
         c.nb = local / mte;
         const int mt = s_tile_off[lo] + (local - c.nb * mte);
         c.valid = true;
@@ -512,8 +525,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-    if (a.mode == GEMM_TAIL_TILES) {
-        if (warp == 2) warp_expert_prefix(s_tile_off, a.E, s_aux, 1, lane);
+    if (a.mode == GEMM_TAIL_TILES || a.mode == GEMM_ODD_EXPERTS) {
+        if (warp == 2)
+            warp_expert_prefix(s_tile_off, a.E, s_aux, a.mode == GEMM_TAIL_TILES ? 1 : 3, lane);
         __syncthreads();
     }
 
@@ -536,9 +550,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         }
         __syncthreads();
     }
-    const bool tails = a.mode == GEMM_TAIL_TILES;
-    const int routed_tiles = (tails ? s_aux[a.E] : a.meta[2]) * a.nb_r;
-    const int shared_tiles = tails ? ((a.mt_s & 1) ? a.nb_s : 0) : a.mt_s * a.nb_s;
+    const bool tails = a.mode == GEMM_TAIL_TILES, odd_only = a.mode == GEMM_ODD_EXPERTS;
+    const int routed_tiles = (tails || odd_only ? s_aux[a.E] : a.meta[2]) * a.nb_r;
+    // the shared expert counts as one more expert: its last m-tile, or all of its
+    // m-tiles, belong here when its m-tile count is odd
+    const int shared_tiles = tails ? ((a.mt_s & 1) ? a.nb_s : 0)
+                                   : odd_only ? ((a.mt_s & 1) ? a.mt_s * a.nb_s : 0)
+                                              : a.mt_s * a.nb_s;
     const int total_tiles = *abort_flag ? 0 : routed_tiles + shared_tiles;
 
     if (warp == 0) {
@@ -668,6 +686,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         tc_fence_after();
         tmem_dealloc(tmem_base, GEMM_TMEM_COLS);
     }
+    // Launched with programmatic serialization after the pair kernel (which reads
+    // and writes none of this launch's rows), this launch starts on the SMs the
+    // pair kernel frees and does not finish before it: the next kernel on the
+    // stream then sees both.  Without that launch attribute this returns at once.
+    grid_dep_wait();
 }
 
 }  // namespace moe
@@ -692,10 +715,12 @@ namespace moe {
 // both; the eight epilogue warps of the pair release an accumulator on CTA 0's
 // tempty[acc].  An expert with an odd number of m-tiles either leaves its last
 // m-tile to the one-CTA kernel in GEMM_TAIL_TILES mode (as does the shared
-// expert's last m-tile when their count is odd) or, in GEMM_PAIR_PAD mode, runs
-// it here as a pair whose second half has no rows (its MMA rows are wasted).
-// Measured on the prefill configurations, neither beat the one-CTA kernel alone,
-// so these kernels run only on request (moe_debug_set_pair_mode).
+// expert's last m-tile when their count is odd), or, in GEMM_PAIR_PAD mode, runs
+// it here as a pair whose second half has no rows (its MMA rows are wasted), or,
+// in GEMM_EVEN_EXPERTS mode, runs wholly on the one-CTA kernel (GEMM_ODD_EXPERTS)
+// while this kernel takes the experts with an even count.  Measured on the
+// prefill configurations, only the last split beat the one-CTA kernel alone, and
+// only for the down GEMM, where it is the default; gate_up stays on one SM.
 // ---------------------------------------------------------------------------
 constexpr int PAIR_STAGES = 6;
 constexpr int PAIR_A_BYTES = GEMM_BM * GEMM_BK * 2;  // 16 KiB: this CTA's 128 rows
@@ -795,7 +820,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     }
     for (int i = threadIdx.x; i <= a.E; i += blockDim.x) s_tile_off[i] = a.tile_off[i];
     __syncthreads();
-    if (warp == 2) warp_expert_prefix(s_tile_off, a.E, s_pair, pad ? 2 : 0, lane);
+    const bool even_only = a.mode == GEMM_EVEN_EXPERTS;
+    if (warp == 2) warp_expert_prefix(s_tile_off, a.E, s_pair, pad ? 2 : even_only ? 4 : 0, lane);
     tc_fence_before();
     // Both CTAs' barriers are initialised and their TMEM allocated before either
     // CTA's loads, MMAs or arrivals can reach the other.
@@ -805,7 +831,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 
     const uint64_t limit = a.wait_limit_ns;
     const int routed_tiles = s_pair[a.E] * a.nb_r;
-    const int total_tiles = routed_tiles + ((pad ? a.mt_s + 1 : a.mt_s) >> 1) * a.nb_s;
+    const int shared_pairs = even_only ? ((a.mt_s & 1) ? 0 : a.mt_s >> 1)
+                                       : (pad ? a.mt_s + 1 : a.mt_s) >> 1;
+    const int total_tiles = routed_tiles + shared_pairs * a.nb_s;
+    // The one-CTA launch that follows (the other experts' tiles) may start on the
+    // SMs this launch frees as its CTAs finish.
+    grid_dep_launch_dependents();
 
     if (warp == 0) {
         // ------------------------------ TMA producer (both CTAs) ------------------

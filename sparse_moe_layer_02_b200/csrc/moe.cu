@@ -26,9 +26,12 @@ constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;
 constexpr int kDecodeMaxTokens = 256;
 uint64_t g_wait_limit_ns = kDefaultWaitLimitNs;
 int g_never_signal = 0;
-// Prefill expert GEMMs on CTA pairs: -1 (default) and 0 never, 1 full pairs with
-// the odd last m-tiles on the one-CTA kernel, 2 every m-tile in pairs, odd ones
-// with an empty half (a test and tuning hook).
+// Prefill expert GEMMs on CTA pairs: 0 never, 1 full pairs with the odd last
+// m-tiles on the one-CTA kernel, 2 every m-tile in pairs, odd ones with an empty
+// half, 3 the even-count experts on pairs and the odd-count ones on the one-CTA
+// kernel, 4 the same for the down GEMM only; -1 selects kDefaultPairMode (a test
+// and tuning hook).
+constexpr int kDefaultPairMode = 4;
 int g_pair_mode = -1;
 // Test hook: device buffer receiving the router's selection scores s' (null: off).
 float *g_dbg_sp = nullptr;
@@ -373,22 +376,27 @@ int launch_router_tc(const RouterParams &p, int sms, const RtcFuse &fz, bool pdl
     return launch_router_tc_t<8, WF32>(mX, mW, p, clk, fz, pdl, st);
 }
 
+// after_pair: launched right after a pair kernel that touches none of this
+// launch's rows, with programmatic stream serialization, so it fills the SMs the
+// pair kernel frees (the kernel waits for the pair kernel before it exits).
 template <int KIND>
 int launch_gemm(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &a2,
                 const CUtensorMap &a3, const CUtensorMap &a4, const CUtensorMap &a5,
-                const GemmArgs &args, int grid, bool cooperative, cudaStream_t st) {
+                const GemmArgs &args, int grid, bool cooperative, cudaStream_t st,
+                bool after_pair = false) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid, 1, 1);
     cfg.blockDim = dim3(GEMM_THREADS, 1, 1);
     cfg.dynamicSmemBytes = GEMM_SMEM_BYTES;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeCooperative;
     attr[0].val.cooperative = cooperative ? 1 : 0;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<KIND>, a0, a1, a2, a3, a4, a5, args) !=
-        cudaSuccess)
+    cfg.numAttrs = after_pair && !cooperative ? 2 : 1;
+    if (launch_ex(cfg, grouped_gemm_kernel<KIND>, a0, a1, a2, a3, a4, a5, args) != cudaSuccess)
         return MOE_ERR_CUDA;
     return launch_status();
 }
@@ -605,7 +613,7 @@ int moe_debug_never_signal(int on) {
 }
 
 int moe_debug_set_pair_mode(int mode) {
-    if (mode < -1 || mode > 2) return MOE_ERR_ARG;
+    if (mode < -1 || mode > 4) return MOE_ERR_ARG;
     g_pair_mode = mode;
     return MOE_OK;
 }
@@ -872,17 +880,28 @@ int forward_impl(const void *x, const void *gate_up, const void *down, const voi
     }
 
     if ((rc = ensure_gemm_attrs(dev)) != MOE_OK) return rc;
-    // CTA pairs only on request: on the configurations measured (two to four
-    // m-tiles per expert on average) the pair kernels were not faster, because
-    // the odd last m-tiles either waste half an MMA tile or, in their own
-    // launch, stream their experts' weights from HBM a second time.
-    bool pair = g_pair_mode >= 1;
+    // CTA pairs by default for the down GEMM only, split by expert parity (mode
+    // 4): on the configurations measured (two to four m-tiles per expert on
+    // average) that made down 2-5 % faster, while gate_up on pairs was as often
+    // slower as faster.  Splitting an expert's m-tiles between the two launches
+    // (mode 1) streams its weights from HBM twice; padding odd m-tiles (mode 2)
+    // wastes half an MMA tile.
+    const int pair_mode = g_pair_mode < 0 ? kDefaultPairMode : g_pair_mode;
+    bool pair = pair_mode >= 1;
     if (pair) {
         if ((rc = ensure_pair_attrs(dev)) != MOE_OK) return rc;
         pair = dev->pair_max_clusters > 0;
     }
     // padded pairs take every m-tile (no one-CTA launch); only if pairs can run
-    const bool pad = pair && g_pair_mode == 2;
+    const bool pad = pair && pair_mode == 2;
+    // modes 3 and 4: the experts with an even m-tile count (and the shared expert
+    // if its count is even) run wholly on pairs, the others wholly on the one-CTA
+    // kernel, so no expert's weights are streamed by both launches; mode 4 does
+    // this for the down GEMM only and runs gate_up on the one-CTA kernel
+    const bool by_parity = pair && (pair_mode == 3 || pair_mode == 4);
+    const bool pair_gu = pair && pair_mode != 4;
+    const int pair_tiles_mode = pad ? GEMM_PAIR_PAD : by_parity ? GEMM_EVEN_EXPERTS : GEMM_ALL_TILES;
+    const int rest_tiles_mode = by_parity ? GEMM_ODD_EXPERTS : GEMM_TAIL_TILES;
     CUtensorMap mx_perm, mgu, mx, msg, msu, mh_perm, mdn, mh_sh, msd, mdn2, msd2;
     bool ok = make_map(&mx_perm, x_perm, D, L.rows_max, D, 128) &&
               make_map(&mgu, gate_up, D, (uint64_t)E * 2 * d_moe, D, 128) &&
@@ -927,19 +946,20 @@ int forward_impl(const void *x, const void *gate_up, const void *down, const voi
     g.ld_s = d_sh;
     g.ncols_s = d_sh;
     int max_tiles = mt_r_max * g.nb_r + mt_s * g.nb_s;
-    if (pair) {
+    g.mode = GEMM_ALL_TILES;
+    if (pair_gu) {
         const int nbm = std::max(g.nb_r, g.nb_s);
-        g.mode = pad ? GEMM_PAIR_PAD : GEMM_ALL_TILES;
+        g.mode = pair_tiles_mode;
         rc = launch_gemm_pair<GEMM_GATE_UP>(mx_perm, mgu, mx, msg, msu, mx, g,
                                             std::min(dev->pair_max_clusters,
                                                      std::max(1, pair_bound_mt * nbm)), st);
         if (rc != MOE_OK) return rc;
-        g.mode = GEMM_TAIL_TILES;
-        max_tiles = tail_bound_mt * nbm;
+        g.mode = rest_tiles_mode;
+        if (!by_parity) max_tiles = tail_bound_mt * nbm;
     }
     if (!pad) {
         rc = launch_gemm<GEMM_GATE_UP>(mx_perm, mgu, mx, msg, msu, mx, g,
-                                       std::min(dev->sms, max_tiles), false, st);
+                                       std::min(dev->sms, max_tiles), false, st, pair_gu);
         if (rc != MOE_OK) return rc;
     }
     prof.mark();
@@ -966,17 +986,17 @@ int forward_impl(const void *x, const void *gate_up, const void *down, const voi
     if (!make_map_out(&mslot, slot, D, L.rows_max, D)) return MOE_ERR_CUDA;
     max_tiles = mt_r_max * g.nb_r + mt_s * g.nb_s;
     if (pair) {
-        g.mode = pad ? GEMM_PAIR_PAD : GEMM_ALL_TILES;
+        g.mode = pair_tiles_mode;
         rc = launch_gemm_pair<GEMM_DOWN>(mh_perm, mdn2, mh_sh, msd2, msd2, mslot, g,
                                          std::min(dev->pair_max_clusters,
                                                   std::max(1, pair_bound_mt * g.nb_r)), st);
         if (rc != MOE_OK) return rc;
-        g.mode = GEMM_TAIL_TILES;
-        max_tiles = tail_bound_mt * g.nb_r;
+        g.mode = rest_tiles_mode;
+        if (!by_parity) max_tiles = tail_bound_mt * g.nb_r;
     }
     if (!pad) {
         rc = launch_gemm<GEMM_DOWN>(mh_perm, mdn, mh_sh, msd, msd, mslot, g,
-                                    std::min(dev->sms, max_tiles), false, st);
+                                    std::min(dev->sms, max_tiles), false, st, pair);
         if (rc != MOE_OK) return rc;
     }
     prof.mark();

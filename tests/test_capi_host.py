@@ -126,7 +126,7 @@ def test_layer_call_rejects_bad_arguments_before_any_launch():
 
 def test_debug_hooks_reject_bad_arguments():
     lib = moe.load_library()
-    assert lib.moe_debug_set_pair_mode(3) == -1
+    assert lib.moe_debug_set_pair_mode(5) == -1
     assert lib.moe_debug_set_pair_mode(-2) == -1
     assert lib.moe_debug_set_pair_mode(-1) == 0
     assert lib.moe_debug_capture_scores(8, 16) == -1      # misaligned buffer

@@ -329,12 +329,12 @@ def test_pair_gemms_match_oracle_and_single_cta(case):
     w = torch.from_numpy(orc["w"]).float().to(DEV)
     ys = {}
     try:
-        for mode in (1, 2, 0):
+        for mode in (1, 2, 3, 4, 0):
             moe.moe_debug_set_pair_mode(mode)
             ys[mode] = _gpu_forward(d, idx, w)
     finally:
         moe.moe_debug_set_pair_mode(-1)
-    for mode in (1, 2):
+    for mode in (1, 2, 3, 4):
         err = rel_err(ys[mode].float().cpu().numpy(), y_ref)
         print(case, mode, err)
         assert err["finite"] and err["max_rel"] <= Y_TOL[cfg.dtype]
@@ -350,12 +350,13 @@ def test_pair_gemms_full_size_equal_single_cta(name):
                             cfg.norm_topk_prob, cfg.alpha)
     ys = {}
     try:
-        for mode in (1, 2, 0):
+        for mode in (1, 2, 3, 4, 0):
             moe.moe_debug_set_pair_mode(mode)
             ys[mode] = _gpu_forward(inp, idx, w)
     finally:
         moe.moe_debug_set_pair_mode(-1)
-    assert torch.equal(ys[1], ys[0]) and torch.equal(ys[2], ys[0])
+    for mode in (1, 2, 3, 4):
+        assert torch.equal(ys[mode], ys[0]), mode
 
 
 # ----------------------------------------------------------------------------- full size
