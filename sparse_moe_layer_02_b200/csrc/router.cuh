@@ -67,16 +67,34 @@ __device__ __forceinline__ uint32_t warp_pick(uint32_t key, uint32_t id) {
     return __reduce_min_sync(0xffffffffu, key == m ? id : 0xffffffffu);
 }
 
+// The float of an order_key (key 0, a NaN's, reads as -inf: never preferred).
+__device__ __forceinline__ float key_value(uint32_t key) {
+    if (key == 0u) return -INFINITY;
+    return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
+}
+
+// Each lane's correction bias for its experts lane, lane + 32, ... (0 past E),
+// loaded once per warp before its tokens.
+template <int EV>
+__device__ __forceinline__ void load_bias(const RouterParams &p, int lane, float (&bv)[EV]) {
+#pragma unroll
+    for (int v = 0; v < EV; ++v) {
+        const int e = lane + 32 * v;
+        bv[v] = e < p.E ? p.b[e] : 0.f;
+    }
+}
+
 // Selection for one token by one warp ("GLM-4.5 Group Router", How it works):
 // lane l holds the fp32 logits of experts l, l+32, ...  s = sigmoid(r),
 // s' = s + b; with n_group > 1 a group scores the sum of its two largest s' and
 // the topk_group best groups are kept (others are -inf); the k largest s' among
 // the kept experts are chosen (ties to the lower id) and their weights are
 // alpha * s / (sum of the chosen s + 1e-20), or alpha * s without normalisation.
-// sp_w is a per-warp scratch row of 32 * ROUTER_MAXV floats in shared memory.
+// sp_w is a per-warp scratch row of 32 * ROUTER_MAXV floats in shared memory; bv
+// the lane's bias values (load_bias).
 template <int EV>
 __device__ __forceinline__ void router_select(const RouterParams &p, int t, const float (&logit)[EV],
-                                              float *sp_w, int lane) {
+                                              const float (&bv)[EV], float *sp_w, int lane) {
     const int E = p.E, G = p.G, m = E / G;
     float s[EV], sp[EV];
 #pragma unroll
@@ -86,13 +104,39 @@ __device__ __forceinline__ void router_select(const RouterParams &p, int t, cons
         sp[v] = -INFINITY;
         if (e < E) {
             s[v] = 1.0f / (1.0f + expf(-logit[v]));
-            sp[v] = s[v] + p.b[e];
+            sp[v] = s[v] + bv[v];
             if (p.dbg_sp) p.dbg_sp[(size_t)t * E + e] = sp[v];
         }
     }
     // Candidate mask over this lane's experts (bit v).
     uint32_t cand = 0;
-    if (G > 1) {
+    if (G > 1 && m == 32 && E % 32 == 0) {
+        // Group g is exactly the slot v = g of every lane: its two largest s'
+        // (equal values both count) by warp reductions on order keys, in
+        // registers.  The same values as the scan below, so the same sum.
+        float gs[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+        for (int g = 0; g < EV; ++g) {
+            if (g < G) {
+                const uint32_t k1 = order_key(sp[g]);
+                const uint32_t m1 = __reduce_max_sync(0xffffffffu, k1);
+                const uint32_t holder = __reduce_min_sync(0xffffffffu, k1 == m1 ? (uint32_t)lane : 32u);
+                const uint32_t m2 = __reduce_max_sync(0xffffffffu, (uint32_t)lane == holder ? 0u : k1);
+                const float score = key_value(m1) + key_value(m2);
+                if (lane == g) gs[0] = score;
+            }
+        }
+        uint64_t kept = 0;
+        const uint32_t gk = order_key(gs[0]);
+        for (int r = 0; r < p.tg; ++r) {
+            const bool mine = lane < G && !((kept >> lane) & 1ull);
+            const uint32_t win = warp_pick(mine ? gk : 0u, mine ? (uint32_t)lane : 0xffffffffu);
+            if (win < 64u) kept |= 1ull << win;
+        }
+#pragma unroll
+        for (int v = 0; v < EV; ++v)
+            if (lane + 32 * v < E && ((kept >> v) & 1ull)) cand |= 1u << v;
+    } else if (G > 1) {
 #pragma unroll
         for (int v = 0; v < EV; ++v)
             if (lane + 32 * v < E) sp_w[lane + 32 * v] = sp[v];
@@ -319,6 +363,8 @@ __global__ void __launch_bounds__(ROUTER_THREADS)
     const int j = rank + ROUTER_CL * warp; // token of this warp (32 = CL * 4 tokens per cluster)
     const int t = t0 + j;
     if (warp < ROUTER_TM / ROUTER_CL && t < p.N) {
+        float bv[EV];
+        load_bias<EV>(p, lane, bv);
         float logit[EV];
 #pragma unroll
         for (int v = 0; v < EV; ++v) {
@@ -333,7 +379,7 @@ __global__ void __launch_bounds__(ROUTER_THREADS)
             }
             logit[v] = r;
         }
-        router_select<EV>(p, t, logit, spbuf + warp * ROUTER_MAXV * 32, lane);
+        router_select<EV>(p, t, logit, bv, spbuf + warp * ROUTER_MAXV * 32, lane);
     }
     cluster.sync(); // keep this CTA's partials alive until every reader is done
 }

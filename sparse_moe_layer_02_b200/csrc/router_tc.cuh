@@ -353,36 +353,59 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
     // ---- sum the cluster's partial logits and select: one warp per token -------
     // Token j of the block goes to CTA j % CLK, so a small batch spreads over the
     // whole cluster.  A lane loads the partials of its experts from every CTA of
-    // the cluster (VB expert slots x CLK ranks in flight) before it adds any, and
-    // adds them in rank order (deterministic).
+    // the cluster before it adds any (all of them when CLK <= 4, else VB expert
+    // slots x CLK ranks at a time), and adds them in rank order (deterministic).
     constexpr int VB = EV < 4 ? EV : 4;
+    float bv[EV];
+    load_bias<EV>(p, lane, bv);
     for (int jl = warp; rank + CLK * jl < RTC_BM; jl += RTC_THREADS / 32) {
         const int j = rank + CLK * jl;
         const int t = t0 + j;
         if (t >= p.N) break;
         float logit[EV];
+        if (CLK <= 4) {
+            float pv[EV][4];
 #pragma unroll
-        for (int v0 = 0; v0 < EV; v0 += VB) {
-            float pv[VB][RTC_MAX_CLK];
-#pragma unroll
-            for (int c = 0; c < RTC_MAX_CLK; ++c) {
+            for (int c = 0; c < 4; ++c) {
                 const float *src = c < CLK ? cluster.map_shared_rank(part, c) + j * RTC_PART_LD : nullptr;
 #pragma unroll
-                for (int v = 0; v < VB; ++v) {
-                    const int e = lane + 32 * (v0 + v);
+                for (int v = 0; v < EV; ++v) {
+                    const int e = lane + 32 * v;
                     pv[v][c] = (c < CLK && e < E) ? src[e] : 0.f;
                 }
             }
 #pragma unroll
-            for (int v = 0; v < VB; ++v) {
+            for (int v = 0; v < EV; ++v) {
                 float r = 0.f;
 #pragma unroll
-                for (int c = 0; c < RTC_MAX_CLK; ++c)
+                for (int c = 0; c < 4; ++c)
                     if (c < CLK) r += pv[v][c];
-                logit[v0 + v] = r;
+                logit[v] = r;
+            }
+        } else {
+#pragma unroll
+            for (int v0 = 0; v0 < EV; v0 += VB) {
+                float pv[VB][RTC_MAX_CLK];
+#pragma unroll
+                for (int c = 0; c < RTC_MAX_CLK; ++c) {
+                    const float *src = c < CLK ? cluster.map_shared_rank(part, c) + j * RTC_PART_LD : nullptr;
+#pragma unroll
+                    for (int v = 0; v < VB; ++v) {
+                        const int e = lane + 32 * (v0 + v);
+                        pv[v][c] = (c < CLK && e < E) ? src[e] : 0.f;
+                    }
+                }
+#pragma unroll
+                for (int v = 0; v < VB; ++v) {
+                    float r = 0.f;
+#pragma unroll
+                    for (int c = 0; c < RTC_MAX_CLK; ++c)
+                        if (c < CLK) r += pv[v][c];
+                    logit[v0 + v] = r;
+                }
             }
         }
-        router_select<EV>(p, t, logit, spbuf + warp * ROUTER_MAXV * 32, lane);
+        router_select<EV>(p, t, logit, bv, spbuf + warp * ROUTER_MAXV * 32, lane);
     }
     cluster.sync(); // partials stay alive until every reader is done
     if (warp == 1) {

@@ -88,23 +88,27 @@ def test_router_bias_reorders_selection_but_not_weights():
     assert rep["unexplained"] == 0 and rep["max_w_err_over_alpha"] <= W_TOL
 
 
+@pytest.mark.parametrize("E", [32, 128])
 @pytest.mark.parametrize("x_dtype", [torch.bfloat16, torch.float32])
-def test_router_exact_ties_go_to_the_lower_index(x_dtype):
+def test_router_exact_ties_go_to_the_lower_index(x_dtype, E):
     """Exact ties, decided the same way on both sides: every expert has a twin with
     an identical router row and bias (so bitwise-equal logits on the GPU and equal
     scores in the oracle), and groups 1 and 3 copy groups 0 and 2 (equal group
     scores; one group is kept, so a group tie sits at the boundary).  Lower ids and
     lower groups win, so the ids must equal the oracle's exactly, order included,
-    with no near-tie allowance."""
-    cfg = CONFIGS["skew_grouped"].with_(N=256, D=256, E=32, n_group=4, topk_group=1, k=3,
+    with no near-tie allowance.  Groups of 8 experts take the shared-memory group
+    scan; groups of 32 the warp-reduction path (a group is one expert slot of
+    every lane), where each group's two largest scores are equal twins."""
+    cfg = CONFIGS["skew_grouped"].with_(N=256, D=256, E=E, n_group=4, topk_group=1, k=3,
                                         skew=False)
+    m = E // 4
     x, wg, b, _ = router_inputs(cfg, seed=17, device=DEV)
     x = x.to(x_dtype)
     wg = wg.clone()
     b = b.clone()
-    for g in (1, 3):                     # group g copies group g - 1 (8 experts each)
-        wg[8 * g:8 * g + 8] = wg[8 * (g - 1):8 * g]
-        b[8 * g:8 * g + 8] = b[8 * (g - 1):8 * g]
+    for g in (1, 3):                     # group g copies group g - 1 (m experts each)
+        wg[m * g:m * g + m] = wg[m * (g - 1):m * g]
+        b[m * g:m * g + m] = b[m * (g - 1):m * g]
     wg[1::2] = wg[0::2]                  # every odd expert copies its even neighbour
     b[1::2] = b[0::2]
     W_g = wg.to(torch.bfloat16) if x_dtype == torch.bfloat16 else wg
@@ -117,12 +121,14 @@ def test_router_exact_ties_go_to_the_lower_index(x_dtype):
     # the even group of each tied pair kept
     gi = idx.cpu().numpy()
     assert any((e ^ 1) not in row for row in gi for e in row)
-    assert set((gi // 8).ravel().tolist()) <= {0, 2}
+    assert set((gi // m).ravel().tolist()) <= {0, 2}
     assert np.max(np.abs(w.cpu().double().numpy() - orc["w"])) / cfg.alpha <= W_TOL
 
 
 @pytest.mark.parametrize("E,G,tg,k", [(64, 8, 3, 6), (512, 1, 1, 8), (288, 1, 1, 8),
-                                      (256, 64, 8, 16), (160, 1, 1, 1)])
+                                      (256, 64, 8, 16), (160, 1, 1, 1),
+                                      # groups of 32 experts (warp-reduction group scores)
+                                      (256, 8, 4, 8), (128, 4, 2, 6)])
 def test_router_shapes(E, G, tg, k):
     cfg = CONFIGS["glm5_prefill"].with_(N=333, D=264, E=E, n_group=G, topk_group=tg, k=k)
     x, wg, b, _ = router_inputs(cfg, seed=E + k, device=DEV)
@@ -134,7 +140,8 @@ def test_router_shapes(E, G, tg, k):
 
 
 @pytest.mark.parametrize("E,G,tg,k,D", [(64, 8, 3, 6, 264), (192, 1, 1, 8, 328), (160, 1, 1, 8, 264),
-                                        (208, 1, 1, 8, 264), (48, 4, 2, 4, 4096)])
+                                        (208, 1, 1, 8, 264), (48, 4, 2, 4, 4096),
+                                        (128, 4, 2, 6, 264)])
 def test_router_fp32_matrix_shapes(E, G, tg, k, D):
     # bf16 tokens with an fp32 router matrix: the tensor-core path splits W_g into
     # three bf16 parts (E <= 192), larger E use the CUDA-core path.
